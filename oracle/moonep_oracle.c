@@ -1,0 +1,375 @@
+/*
+ * moonep_oracle.c -- CPU oracle for the balanced expert-parallel hot path
+ * (planner, dispatch, combine, weight prefetch, grad-slot reduction).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may call, link or
+ * load this file; only the tests, the package's smoke check and the
+ * benchmark's CPU-baseline leg do.  It shares no code, header, table or
+ * helper with the CUDA path.  It is deliberately plain and slow: one thread,
+ * no blocking, no fusion, every step in the order the rule states it.
+ * Floating point is accumulated in fp64 and rounded once at the end.
+ *
+ * Sources (web pages about MoonEP; "README" is the project's GitHub README,
+ * "MTP" the MarkTechPost article "Moonshot AI Open-Sources MoonEP: A Perfectly
+ * Balanced Expert Parallelism Library for MoE Training"):
+ *   - maxvio = max_e(T_e / T_bar) - 1, T_bar the per-expert count under perfect
+ *     balance: README section "Performance"; MTP, "The problem MoonEP targets".
+ *   - every rank receives exactly S x K token slots: README, intro item 1
+ *     ("Perfect balance"); MTP, "Core idea: dynamic redundant experts".
+ *   - training copies come from at most one remote home group per rank, so
+ *     B = E/R; inference may use B < E/R and then reads overflow experts from
+ *     their home rows: README, "How to set B"; MTP, "Memory contract".
+ *   - rows [0,E) are the home experts, rows [E,E+B) the prefetch slots,
+ *     cu_seqlens[E+B] the padded end offset of each row: README, "Weight
+ *     buffer" and "dispatch fwd"; MTP, "Memory contract".
+ *   - dispatch writes each token straight into its expert-grouped slot and
+ *     returns the route weight per slot; combine gathers the K rows back and
+ *     weights them: README, "dispatch fwd", "combine fwd", "dispatch bwd".
+ *   - reduce_grad adds every rank's slot gradients of a home expert into its
+ *     parameter gradient and zeroes the consumed slots: README, "Grad buffer";
+ *     MTP, "Memory contract".
+ *
+ * The pages name the invariants but print no planning rule.  The rule below is
+ * this library's fixed reading; every choice the pages leave open is marked
+ * [reading].
+ *
+ * Plan rule.  G = E/R experts per home group, C = S*K slots per rank,
+ * home(e) = e / G.
+ *  1. cnt[r][e] = picks of expert e on source rank r; T_e = sum_r cnt[r][e];
+ *     L_h = sum of T_e over group h; maxvio = max_e T_e / (R*S*K/E) - 1.
+ *  2. The group sequence of home rank h lists every pick (r,t,k) whose expert
+ *     lies in group h, ordered by expert, then source rank, then token.
+ *     [reading]
+ *  3. Walker/Vose alias chain over the loads L_h: the lowest-numbered
+ *     under-loaded rank takes C - cur from the lowest-numbered over-loaded
+ *     rank; a donor that drops below C is served next.  Each rank receives
+ *     from at most one donor; there are at most R-1 donations.  [reading]
+ *  4. A donor keeps the prefix of its group sequence; its donations take
+ *     consecutive ranges after it, in the order they were made.  [reading]
+ *  5. On rank s: row e (e in group s) holds the kept picks of e; the distinct
+ *     experts s received, in ascending id, take slots b = 0,1,.. (row E+b);
+ *     past B they go to row e itself (inference overflow).  [reading]
+ *  6. Within a row, picks keep group-sequence order.  Rows are padded to a
+ *     multiple of tp (empty rows stay empty); cu_seqlens is the inclusive
+ *     running sum of the padded lengths over the E+B rows.  [reading]
+ *  7. NvS = roundup(C + 2*G*(tp-1), tp): at most G home rows plus G received
+ *     rows are non-empty.  [reading]
+ *  8. dst[r,t,k] = dest_rank*NvS + row start + position inside the row.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* status bits (kept numerically equal to the public header's by the tests) */
+#define ORC_BAD_EXPERT 1
+#define ORC_DUP_EXPERT 2
+#define ORC_COUNT_MISMATCH 4
+#define ORC_BAD_ARGS 256
+
+static int64_t pad_up(int64_t n, int64_t tp) { return (n + tp - 1) / tp * tp; }
+
+int64_t oracle_nvs(int S, int K, int E, int R, int tp)
+{
+    int64_t C = (int64_t)S * K, G = E / R;
+    return pad_up(C + 2 * G * (tp - 1), tp);
+}
+
+/* ---- bf16 <-> double ------------------------------------------------------ */
+
+static double bf16_to_double(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return (double)f;
+}
+
+/* Round x to the nearest bf16 value, ties to even, directly from fp64 (no
+ * intermediate fp32 rounding).  bf16 keeps 8 significant bits and the fp32
+ * exponent range; below 2^-126 its spacing is fixed at 2^-133. */
+uint16_t oracle_double_to_bf16(double x)
+{
+    if (isnan(x)) return 0x7FC0;
+    uint16_t sign = signbit(x) ? 0x8000 : 0;
+    double ax = fabs(x);
+    if (ax == 0.0) return sign;
+    int ex;
+    frexp(ax, &ex); /* ax = m * 2^ex, m in [0.5, 1) */
+    int lsb = ex - 8;
+    if (lsb < -133) lsb = -133;
+    double q = ldexp(1.0, lsb);
+    double v = nearbyint(ax / q) * q; /* default rounding: to nearest, ties to even */
+    float f = (float)v;               /* exact, or +inf past the bf16 range */
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    return (uint16_t)(sign | ((u >> 16) & 0x7FFF));
+}
+
+/* ---- plan --------------------------------------------------------------- */
+
+/*
+ * Inputs: topk [R,S,K] int32 (expert ids), tpe [R,E] int32 or NULL (the
+ * router's local counts, checked against the picks).  mode 0 = training
+ * (B >= E/R), 1 = inference.
+ * Outputs (caller-allocated): dst [R,S,K], cu_seqlens [R,E+B],
+ * row_counts [R,E+B], slot_expert [R,B] (-1 = unused), counts [R,E],
+ * maxvio [1], assign [R,4] = {kept, donor group or -1, received start in the
+ * donor's group sequence, received length}.
+ * Returns 0 or a bitmask of ORC_* errors; on error the outputs other than
+ * counts are not written.
+ */
+int oracle_plan(int R, int S, int K, int E, int B, int tp, int mode,
+                const int32_t *topk, const int32_t *tpe,
+                int32_t *dst, int32_t *cu_seqlens, int32_t *row_counts,
+                int32_t *slot_expert, int32_t *counts, float *maxvio,
+                int32_t *assign)
+{
+    if (R < 1 || S < 1 || K < 1 || E < 1 || E % R || K > E || B < 0 || tp < 1)
+        return ORC_BAD_ARGS;
+    const int G = E / R;
+    if (mode == 0 && B < G) return ORC_BAD_ARGS;
+    const int64_t C = (int64_t)S * K;
+    const int NR = E + B; /* rows per rank */
+    const int64_t NvS = oracle_nvs(S, K, E, R, tp);
+    int status = 0;
+
+    /* validation: ids in [0,E), no expert twice within one token */
+    for (int r = 0; r < R; r++)
+        for (int t = 0; t < S; t++) {
+            const int32_t *tok = topk + ((int64_t)r * S + t) * K;
+            for (int k = 0; k < K; k++) {
+                int e = tok[k];
+                if (e < 0 || e >= E) { status |= ORC_BAD_EXPERT; continue; }
+                for (int k2 = 0; k2 < k; k2++)
+                    if (tok[k2] == e) status |= ORC_DUP_EXPERT;
+            }
+        }
+
+    /* step 1: counts over the valid picks */
+    memset(counts, 0, sizeof(int32_t) * (size_t)R * E);
+    for (int r = 0; r < R; r++)
+        for (int64_t i = 0; i < C; i++) {
+            int e = topk[(int64_t)r * C + i];
+            if (e >= 0 && e < E) counts[(int64_t)r * E + e]++;
+        }
+    if (tpe)
+        for (int64_t i = 0; i < (int64_t)R * E; i++)
+            if (tpe[i] != counts[i]) status |= ORC_COUNT_MISMATCH;
+    if (status) return status;
+
+    int64_t *T = calloc(E, sizeof(int64_t));
+    int64_t *L = calloc(R, sizeof(int64_t));
+    for (int e = 0; e < E; e++) {
+        for (int r = 0; r < R; r++) T[e] += counts[(int64_t)r * E + e];
+        L[e / G] += T[e];
+    }
+    int64_t maxT = 0;
+    for (int e = 0; e < E; e++)
+        if (T[e] > maxT) maxT = T[e];
+    double Tbar = (double)((int64_t)R * S * K) / (double)E;
+    *maxvio = (float)((double)maxT / Tbar - 1.0);
+
+    /* step 3: alias chain.  small is a deque (push to the front when a donor
+     * falls below C), large a queue, both seeded in ascending rank order. */
+    int64_t *cur = malloc(sizeof(int64_t) * R);
+    int *smallq = malloc(sizeof(int) * 2 * R), sh = R, st = R; /* [sh, st) */
+    int *largeq = malloc(sizeof(int) * R), lh = 0, lt = 0;
+    int *don_from = malloc(sizeof(int) * R), *don_to = malloc(sizeof(int) * R);
+    int64_t *don_amt = malloc(sizeof(int64_t) * R);
+    int ndon = 0;
+    for (int h = 0; h < R; h++) {
+        cur[h] = L[h];
+        if (L[h] < C) smallq[st++] = h;
+        if (L[h] > C) largeq[lt++] = h;
+    }
+    while (sh < st) {
+        int s = smallq[sh++];
+        int l = largeq[lh]; /* exists: sum(cur) == R*C */
+        int64_t d = C - cur[s];
+        don_from[ndon] = l; don_to[ndon] = s; don_amt[ndon] = d; ndon++;
+        cur[s] = C;
+        cur[l] -= d;
+        if (cur[l] < C) { lh++; smallq[--sh] = l; }
+        else if (cur[l] == C) lh++;
+    }
+
+    /* step 4: kept prefix and donated ranges of each donor's group sequence */
+    int64_t *keep = malloc(sizeof(int64_t) * R);
+    int64_t *don_start = malloc(sizeof(int64_t) * R);
+    for (int h = 0; h < R; h++) {
+        keep[h] = L[h];
+        for (int j = 0; j < ndon; j++)
+            if (don_from[j] == h) keep[h] -= don_amt[j];
+    }
+    for (int h = 0; h < R; h++) {
+        int64_t next = keep[h];
+        for (int j = 0; j < ndon; j++)
+            if (don_from[j] == h) { don_start[j] = next; next += don_amt[j]; }
+    }
+    for (int s = 0; s < R; s++) {
+        assign[s * 4 + 0] = (int32_t)keep[s];
+        assign[s * 4 + 1] = -1;
+        assign[s * 4 + 2] = 0;
+        assign[s * 4 + 3] = 0;
+    }
+    for (int j = 0; j < ndon; j++) {
+        int s = don_to[j];
+        assign[s * 4 + 1] = don_from[j];
+        assign[s * 4 + 2] = (int32_t)don_start[j];
+        assign[s * 4 + 3] = (int32_t)don_amt[j];
+    }
+
+    /* start of each expert's run inside its group sequence */
+    int64_t *estart = calloc(E, sizeof(int64_t));
+    for (int e = 0; e < E; e++)
+        estart[e] = (e % G == 0) ? 0 : estart[e - 1] + T[e - 1];
+
+    /* step 5: rows of every rank */
+    memset(row_counts, 0, sizeof(int32_t) * (size_t)R * NR);
+    for (int64_t i = 0; i < (int64_t)R * B; i++) slot_expert[i] = -1;
+    for (int s = 0; s < R; s++) {
+        int32_t *n = row_counts + (int64_t)s * NR;
+        for (int e = s * G; e < (s + 1) * G; e++) {
+            int64_t lo = estart[e], hi = estart[e] + T[e];
+            if (hi > keep[s]) hi = keep[s];
+            if (hi > lo) n[e] = (int32_t)(hi - lo);
+        }
+        int h = assign[s * 4 + 1];
+        if (h >= 0) {
+            int64_t a = assign[s * 4 + 2], b = a + assign[s * 4 + 3];
+            int q = 0;
+            for (int e = h * G; e < (h + 1) * G; e++) {
+                int64_t lo = estart[e] > a ? estart[e] : a;
+                int64_t hi = estart[e] + T[e] < b ? estart[e] + T[e] : b;
+                if (hi <= lo) continue;
+                if (q < B) {
+                    slot_expert[(int64_t)s * B + q] = e;
+                    n[E + q] += (int32_t)(hi - lo);
+                } else {
+                    n[e] += (int32_t)(hi - lo); /* overflow: the expert's home row */
+                }
+                q++;
+            }
+        }
+    }
+
+    /* step 6: padded inclusive end offsets */
+    for (int s = 0; s < R; s++) {
+        int64_t run = 0;
+        for (int i = 0; i < NR; i++) {
+            int64_t n = row_counts[(int64_t)s * NR + i];
+            run += n ? pad_up(n, tp) : 0;
+            cu_seqlens[(int64_t)s * NR + i] = (int32_t)run;
+        }
+    }
+
+    /* step 8: walk each group sequence in order and place every pick */
+    int32_t *fill = calloc((size_t)R * NR, sizeof(int32_t));
+    for (int h = 0; h < R; h++) {
+        int64_t g = 0;
+        for (int e = h * G; e < (h + 1) * G; e++)
+            for (int r = 0; r < R; r++)
+                for (int t = 0; t < S; t++)
+                    for (int k = 0; k < K; k++) {
+                        int64_t idx = ((int64_t)r * S + t) * K + k;
+                        if (topk[idx] != e) continue;
+                        int dest = h, row = e;
+                        if (g >= keep[h]) {
+                            for (int j = 0; j < ndon; j++)
+                                if (don_from[j] == h && g >= don_start[j] &&
+                                    g < don_start[j] + don_amt[j])
+                                    dest = don_to[j];
+                            for (int b = 0; b < B; b++)
+                                if (slot_expert[(int64_t)dest * B + b] == e) row = E + b;
+                        }
+                        int64_t ri = (int64_t)dest * NR + row;
+                        int64_t n = row_counts[ri];
+                        int64_t row_start = cu_seqlens[ri] - pad_up(n, tp);
+                        dst[idx] = (int32_t)(dest * NvS + row_start + fill[ri]);
+                        fill[ri]++;
+                        g++;
+                    }
+    }
+
+    free(fill); free(estart); free(don_start); free(keep); free(don_amt);
+    free(don_to); free(don_from); free(largeq); free(smallq); free(cur);
+    free(L); free(T);
+    return 0;
+}
+
+/* ---- dispatch / combine --------------------------------------------------- */
+
+/* buf[dst[r,t,k], :] = hidden[r,t,:]; w_nvs[dst] = w[r,t,k] (both optional). */
+void oracle_dispatch(int R, int S, int K, int H, const int32_t *dst,
+                     const uint16_t *hidden, const float *w, uint16_t *buf, float *w_nvs)
+{
+    for (int r = 0; r < R; r++)
+        for (int t = 0; t < S; t++)
+            for (int k = 0; k < K; k++) {
+                int64_t idx = ((int64_t)r * S + t) * K + k;
+                int64_t d = dst[idx];
+                for (int c = 0; c < H; c++)
+                    buf[d * H + c] = hidden[((int64_t)r * S + t) * H + c];
+                if (w && w_nvs) w_nvs[d] = w[idx];
+            }
+}
+
+/* out[r,t,:] = bf16( sum_k w_nvs[d_k] * y[d_k,:] ), the sum in fp64 and
+ * rounded once; w_nvs NULL = unweighted.  gathered_w[r,t,k] = w_nvs[d_k]. */
+void oracle_combine(int R, int S, int K, int H, const int32_t *dst, const uint16_t *y,
+                    const float *w_nvs, uint16_t *out, float *gathered_w)
+{
+    for (int r = 0; r < R; r++)
+        for (int t = 0; t < S; t++) {
+            const int32_t *d = dst + ((int64_t)r * S + t) * K;
+            for (int c = 0; c < H; c++) {
+                double acc = 0.0;
+                for (int k = 0; k < K; k++) {
+                    double wk = w_nvs ? (double)w_nvs[d[k]] : 1.0;
+                    acc += wk * bf16_to_double(y[(int64_t)d[k] * H + c]);
+                }
+                out[((int64_t)r * S + t) * H + c] = oracle_double_to_bf16(acc);
+            }
+            if (w_nvs && gathered_w)
+                for (int k = 0; k < K; k++)
+                    gathered_w[((int64_t)r * S + t) * K + k] = w_nvs[d[k]];
+        }
+}
+
+/* ---- weight prefetch / grad-slot reduction (one projection per call) ------ */
+
+/* pool[s,:] = W[slot_expert[s],:] for every used slot s of the R*B slots. */
+void oracle_prefetch(int R, int B, int64_t HHp, const int32_t *slot_expert,
+                     const uint16_t *W, uint16_t *pool)
+{
+    for (int64_t s = 0; s < (int64_t)R * B; s++) {
+        int e = slot_expert[s];
+        if (e < 0) continue;
+        memcpy(pool + s * HHp, W + (int64_t)e * HHp, sizeof(uint16_t) * (size_t)HHp);
+    }
+}
+
+/* For each expert e: G[e] += sum of RB[s] over the slots s holding e, in
+ * ascending slot order (s = r*B + b), the sum in fp64 rounded once to fp32;
+ * then every consumed slot is set to +0.0.  Unused slots are untouched. */
+void oracle_reduce_grad(int R, int B, int E, int64_t HHp, const int32_t *slot_expert,
+                        float *Gr, float *RB)
+{
+    int64_t nslot = (int64_t)R * B;
+    int64_t *holders = malloc(sizeof(int64_t) * (size_t)(nslot > 0 ? nslot : 1));
+    for (int e = 0; e < E; e++) {
+        int64_t nh = 0;
+        for (int64_t s = 0; s < nslot; s++)
+            if (slot_expert[s] == e) holders[nh++] = s; /* ascending slot order */
+        if (nh == 0) continue;
+        for (int64_t i = 0; i < HHp; i++) {
+            double acc = (double)Gr[(int64_t)e * HHp + i];
+            for (int64_t j = 0; j < nh; j++) acc += (double)RB[holders[j] * HHp + i];
+            Gr[(int64_t)e * HHp + i] = (float)acc;
+        }
+        for (int64_t j = 0; j < nh; j++)
+            for (int64_t i = 0; i < HHp; i++) RB[holders[j] * HHp + i] = 0.0f;
+    }
+    free(holders);
+}
