@@ -1,0 +1,215 @@
+/*
+ * moonep.h -- C ABI of the balanced expert-parallel (EP) hot path, one B200.
+ *
+ * The operations are those of MoonEP ("MoonEP: A Perfectly Balanced Expert
+ * Parallelism Library via Dynamic Redundant Experts", the project's GitHub
+ * README, and the MarkTechPost article "Moonshot AI Open-Sources MoonEP").
+ * An EP group of R ranks is emulated on one GPU: every per-rank tensor carries
+ * a leading [R] dimension and the R partitions live in one device allocation.
+ * A remote access of the original design is an offset into that allocation.
+ *
+ * Notation (README, "Usage > Integration"): S input tokens per rank, K experts
+ * per token, E routed experts in the group, R ranks, B prefetch slots per rank,
+ * H hidden size, H' expert FFN intermediate size, NvS dispatched token slots
+ * per rank (S*K real slots plus the padding of every row), G = E/R experts per
+ * home group.  bf16 tensors are passed as void pointers to 16-bit values.
+ *
+ * Conventions for every call:
+ *  - All tensor arguments are DEVICE pointers on the device that was current
+ *    when the handle was created, row-major and densely packed.  The caller
+ *    owns every tensor, including the plan arrays; the library owns only the
+ *    handle and a small planning workspace inside it.
+ *  - Every call is asynchronous on `stream` (NULL = legacy default stream) and
+ *    never synchronises the host, except moonep_read_status.
+ *  - Return value: MOONEP_OK, or a negative MOONEP_ERR_* for errors detected
+ *    on the host before anything is launched.  Data-dependent errors are found
+ *    on the device and reported as MOONEP_STATUS_* bits in plan->status; every
+ *    later call that takes that plan then does nothing.
+ *  - Calls that share a handle must be ordered on one stream (they share the
+ *    planning workspace).  Calls that overlap on the GPU and write the same
+ *    caller buffers race.
+ */
+#ifndef MOONEP_H
+#define MOONEP_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MOONEP_API __attribute__((visibility("default")))
+#else
+#define MOONEP_API
+#endif
+
+/* Same type as cudaStream_t; declared here so callers need no CUDA header. */
+typedef struct CUstream_st *moonep_stream_t;
+
+/* host-side error codes (return values) */
+#define MOONEP_OK 0
+#define MOONEP_ERR_NULL (-1)   /* a required pointer is NULL */
+#define MOONEP_ERR_CONFIG (-2) /* the configuration is rejected (see moonep_create) */
+#define MOONEP_ERR_ALIGN (-3)  /* a tensor pointer is not 16-byte aligned */
+#define MOONEP_ERR_CUDA (-4)   /* a CUDA runtime call failed (allocation or launch) */
+#define MOONEP_ERR_SIZE (-5)   /* a size argument is outside the supported range */
+
+/* device-side status bits, OR-ed into plan->status */
+#define MOONEP_STATUS_BAD_EXPERT 1     /* an expert id outside [0, E) (e.g. a -1 mask) */
+#define MOONEP_STATUS_DUP_EXPERT 2     /* an expert picked twice by one token */
+#define MOONEP_STATUS_COUNT_MISMATCH 4 /* tokens_per_expert differs from the picks */
+#define MOONEP_STATUS_BAD_PLAN 8       /* a plan index pointed outside its buffer; skipped */
+
+/* Supported ranges (moonep_create checks them). */
+#define MOONEP_MAX_R 64
+#define MOONEP_MAX_E 4096
+#define MOONEP_MAX_K 32
+#define MOONEP_MAX_PROJ 8
+
+/*
+ * Construction parameters; they follow the README's
+ * Buffer(S, H, K, E, num_ep_ranks, num_sms, token_padding, B) ("API guide").
+ *   S, H, K, E, R, B : as in the notation above.  H % 8 == 0 (rows move as
+ *                      16-byte vectors).  E % R == 0.  1 <= K <= min(E, 32).
+ *   token_padding    : every non-empty row is padded to a multiple of it.
+ *   num_sms          : SMs the copy kernels may occupy; 0 = all of them.
+ *   mode             : 0 = training, which needs B >= E/R because copies come
+ *                      from at most one remote home group per rank; 1 =
+ *                      inference, any B >= 0, copied experts past the first B
+ *                      are read from their home rows ("How to set B").
+ */
+typedef struct {
+    int32_t S, H, K, E, R, B, token_padding, num_sms, mode;
+} moonep_config_t;
+
+/*
+ * A plan: caller-owned DEVICE arrays, written by moonep_plan and read by every
+ * other call.  The README keeps the plan ("MoonEPCommPlan") for prefetch,
+ * combine and both backward passes ("dispatch fwd").
+ *   dst         [R,S,K] int32  slot of pick (r,t,k): dest_rank*NvS + row start + position
+ *   cu_seqlens  [R,E+B] int32  inclusive padded end offset of each row of each rank
+ *   row_counts  [R,E+B] int32  real picks per row
+ *   slot_expert [R,B]   int32  expert held by prefetch slot b of rank r, -1 = unused
+ *   counts      [R,E]   int32  picks of expert e made on source rank r
+ *   assign      [R,4]   int32  per rank: picks of its own group it keeps, donor
+ *                              group it takes copies from (-1 none), start and
+ *                              length of the range it takes in that group's
+ *                              sequence
+ *   maxvio      [1]     float  max_e(T_e / T_bar) - 1 ("Performance")
+ *   status      [1]     int32  0 or MOONEP_STATUS_* bits
+ */
+typedef struct {
+    int32_t *dst;
+    int32_t *cu_seqlens;
+    int32_t *row_counts;
+    int32_t *slot_expert;
+    int32_t *counts;
+    int32_t *assign;
+    float *maxvio;
+    int32_t *status;
+} moonep_plan_t;
+
+typedef struct moonep_handle *moonep_handle_t;
+
+/*
+ * Validate cfg and create a handle on the current device; allocates the
+ * planning workspace (cudaMalloc, a few hundred KB).  Rejects (ERR_CONFIG):
+ * E % R != 0, K > E, H % 8 != 0, training with B < E/R, sizes past the
+ * MOONEP_MAX_* limits, R*S*K or R*NvS at or above 2^31.  *out is NULL on error.
+ */
+MOONEP_API int moonep_create(const moonep_config_t *cfg, moonep_handle_t *out);
+
+/* Free the handle and its workspace.  NULL is accepted.  The caller makes sure
+ * no call on the handle is still running on the GPU. */
+MOONEP_API int moonep_destroy(moonep_handle_t h);
+
+/* NvS = roundup(S*K + 2*(E/R)*(token_padding-1), token_padding): the slots of
+ * one rank's static buffer (README notation "NvS").  Negative on a NULL handle. */
+MOONEP_API int64_t moonep_nvs(moonep_handle_t h);
+
+/* Copy the handle's configuration into *out. */
+MOONEP_API int moonep_get_config(moonep_handle_t h, moonep_config_t *out);
+
+/*
+ * Plan one layer: read the router output of all R ranks and write *plan.
+ * README "dispatch fwd" (planning part), "Performance" item 2 (online
+ * planning); the planning rule itself is this library's reading of the pages
+ * (documented in the repository's design notes and in oracle/moonep_oracle.c).
+ *   topk              [R,S,K] int32  expert ids picked by each token
+ *   tokens_per_expert [R,E]   int32  the router's local counts, or NULL; when
+ *                                    given, checked against the picks
+ * Every rank ends with exactly S*K real slots.  Device-side errors: BAD_EXPERT,
+ * DUP_EXPERT, COUNT_MISMATCH (then the other plan arrays are unspecified).
+ */
+MOONEP_API int moonep_plan(moonep_handle_t h, const int32_t *topk, const int32_t *tokens_per_expert,
+                const moonep_plan_t *plan, moonep_stream_t stream);
+
+/*
+ * Fused-permute dispatch (README "dispatch fwd"; "combine bwd" is the same call
+ * on the output gradient with the saved plan): every token row is written
+ * straight into its K expert-grouped slots.
+ *   hidden            [R,S,H]  bf16   token rows
+ *   route_weights     [R,S,K]  fp32   or NULL
+ *   hidden_nvs        [R,NvS,H] bf16  written at the real slots only; padding
+ *                                     slots are left as they were
+ *   route_weights_nvs [R,NvS]  fp32   or NULL; written at the real slots
+ * hidden, hidden_nvs: 16-byte aligned.
+ */
+MOONEP_API int moonep_dispatch(moonep_handle_t h, const moonep_plan_t *plan, const void *hidden,
+                    const float *route_weights, void *hidden_nvs, float *route_weights_nvs,
+                    moonep_stream_t stream);
+
+/*
+ * Combine (README "combine fwd"; "dispatch bwd" calls it with
+ * route_weights_nvs = NULL): out[r,t,:] = bf16(sum_k w_k * y[dst[r,t,k],:]),
+ * accumulated in fp32 in k order, rounded to nearest even.
+ *   hidden_nvs        [R,NvS,H] bf16  expert output y
+ *   route_weights_nvs [R,NvS]   fp32  or NULL for the unweighted sum (w_k = 1)
+ *   out               [R,S,H]   bf16
+ *   gathered_weights  [R,S,K]   fp32  or NULL; = route_weights_nvs[dst]
+ * hidden_nvs, out: 16-byte aligned.
+ */
+MOONEP_API int moonep_combine(moonep_handle_t h, const moonep_plan_t *plan, const void *hidden_nvs,
+                   const float *route_weights_nvs, void *out, float *gathered_weights,
+                   moonep_stream_t stream);
+
+/*
+ * Weight prefetch (README "Weight buffer", "dispatch fwd" prefetch_weight):
+ * for each projection p and each used slot (r,b), pool[p][r][b] = W[p][e] with
+ * e = slot_expert[r][b].  Each expert is read once and written to every slot
+ * holding it.
+ *   weights[p] [E,H,Hp]   bf16  the home experts (rows [0,E) of the pages'
+ *                               [E+B,H,H'] tensor)
+ *   pool[p]    [R,B,H,Hp] bf16  rank r's rows [E,E+B)
+ * 1 <= n_proj <= MOONEP_MAX_PROJ; all pointers 16-byte aligned.
+ */
+MOONEP_API int moonep_prefetch_weight(moonep_handle_t h, const moonep_plan_t *plan, int32_t n_proj,
+                           const void *const *weights, void *const *pool, int64_t Hp,
+                           moonep_stream_t stream);
+
+/*
+ * Grad-slot reduction (README "Grad buffer", "dispatch bwd" reduce_grad): for
+ * each projection and each expert e held by at least one slot,
+ * grads[p][e] += sum of reduce_buffers[p][r][b] over the slots holding e, in
+ * ascending (r,b) order in fp32; then every consumed slot is set to +0.0 for
+ * the next microbatch.  Unused slots are untouched.
+ *   grads[p]          [E,H,Hp]   fp32  the home experts' parameter gradients
+ *   reduce_buffers[p] [R,B,H,Hp] fp32  all ranks' slot gradients
+ * 1 <= n_proj <= MOONEP_MAX_PROJ; all pointers 16-byte aligned.
+ */
+MOONEP_API int moonep_reduce_grad(moonep_handle_t h, const moonep_plan_t *plan, int32_t n_proj,
+                       float *const *grads, float *const *reduce_buffers, int64_t Hp,
+                       moonep_stream_t stream);
+
+/* Read plan->status into *status (host).  Synchronises `stream`. */
+MOONEP_API int moonep_read_status(const moonep_plan_t *plan, int32_t *status, moonep_stream_t stream);
+
+/* Static description of a MOONEP_ERR_* code. */
+MOONEP_API const char *moonep_error_string(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOONEP_H */

@@ -1,0 +1,234 @@
+// C ABI of libmoonep: host-side validation, the handle, and kernel launches.
+// Every entry point is declared and documented in include/moonep.h.
+#include <stdlib.h>
+#include <string.h>
+
+#include "moonep_internal.cuh"
+
+namespace moonep {
+cudaError_t plan_set_smem_limit(size_t bytes);
+cudaError_t weights_set_smem_limit(size_t bytes);
+}  // namespace moonep
+
+using namespace moonep;
+
+struct moonep_handle {
+    moonep_config_t cfg;
+    Dims d;
+    int device;
+    int sms;            // SMs the copy kernels may occupy
+    int grid_dispatch;  // whole waves over those SMs
+    int grid_combine;
+    int grid_weights;
+    void *ws_mem;
+    Workspace ws;
+};
+
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static int fail_cuda(cudaError_t e) {
+    (void)e;
+    return MOONEP_ERR_CUDA;
+}
+
+extern "C" const char *moonep_error_string(int code) {
+    switch (code) {
+        case MOONEP_OK: return "ok";
+        case MOONEP_ERR_NULL: return "a required pointer is NULL";
+        case MOONEP_ERR_CONFIG: return "configuration rejected";
+        case MOONEP_ERR_ALIGN: return "tensor pointer not 16-byte aligned";
+        case MOONEP_ERR_CUDA: return "CUDA runtime call failed";
+        case MOONEP_ERR_SIZE: return "size argument out of the supported range";
+        default: return "unknown moonep error";
+    }
+}
+
+static int64_t nvs_of(const moonep_config_t &c) {
+    const int64_t C = (int64_t)c.S * c.K, G = c.E / c.R, tp = c.token_padding;
+    const int64_t n = C + 2 * G * (tp - 1);
+    return (n + tp - 1) / tp * tp;
+}
+
+static int check_config(const moonep_config_t &c) {
+    if (c.R < 1 || c.R > MOONEP_MAX_R) return MOONEP_ERR_CONFIG;
+    if (c.E < 1 || c.E > MOONEP_MAX_E || c.E % c.R != 0) return MOONEP_ERR_CONFIG;
+    if (c.K < 1 || c.K > MOONEP_MAX_K || c.K > c.E) return MOONEP_ERR_CONFIG;
+    if (c.S < 1 || c.H < 8 || c.H % 8 != 0) return MOONEP_ERR_CONFIG;
+    if (c.B < 0 || c.token_padding < 1 || c.num_sms < 0) return MOONEP_ERR_CONFIG;
+    if (c.mode != 0 && c.mode != 1) return MOONEP_ERR_CONFIG;
+    if (c.mode == 0 && c.B < c.E / c.R) return MOONEP_ERR_CONFIG;
+    if ((int64_t)c.R * c.B > 4096 || c.E + (int64_t)c.B > (int64_t)1 << 20) return MOONEP_ERR_CONFIG;
+    if ((int64_t)c.R * c.S * c.K >= ((int64_t)1 << 31)) return MOONEP_ERR_CONFIG;
+    if (c.token_padding > (1 << 20)) return MOONEP_ERR_CONFIG;
+    if ((int64_t)c.R * nvs_of(c) >= ((int64_t)1 << 31)) return MOONEP_ERR_CONFIG;
+    return MOONEP_OK;
+}
+
+static bool plan_ok(const moonep_plan_t *p) {
+    return p && p->dst && p->cu_seqlens && p->row_counts && p->counts && p->assign && p->maxvio && p->status;
+}
+
+extern "C" int moonep_create(const moonep_config_t *cfg, moonep_handle_t *out) {
+    if (!out) return MOONEP_ERR_NULL;
+    *out = nullptr;
+    if (!cfg) return MOONEP_ERR_NULL;
+    const int rc = check_config(*cfg);
+    if (rc != MOONEP_OK) return rc;
+
+    moonep_handle *h = static_cast<moonep_handle *>(calloc(1, sizeof(moonep_handle)));
+    if (!h) return MOONEP_ERR_CUDA;
+    h->cfg = *cfg;
+    Dims &d = h->d;
+    d.S = cfg->S; d.H = cfg->H; d.K = cfg->K; d.E = cfg->E; d.R = cfg->R; d.B = cfg->B;
+    d.tp = cfg->token_padding; d.mode = cfg->mode;
+    d.G = d.E / d.R;
+    d.nch = (d.S + kChunkTokens - 1) / kChunkTokens;
+    d.NR = d.E + d.B;
+    d.nvs = (int)nvs_of(*cfg);
+
+    cudaError_t e = cudaGetDevice(&h->device);
+    int sms = 0;
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, h->device);
+    if (e != cudaSuccess) { free(h); return fail_cuda(e); }
+    h->sms = (cfg->num_sms > 0 && cfg->num_sms < sms) ? cfg->num_sms : sms;
+
+    const size_t smem = plan_count_smem_bytes(d);
+    if (smem > 227 * 1024) { free(h); return MOONEP_ERR_CONFIG; }
+    if (smem > 48 * 1024 && (e = plan_set_smem_limit(smem)) != cudaSuccess) { free(h); return fail_cuda(e); }
+    const size_t wsmem = sizeof(int32_t) * 3 * (size_t)d.R * d.B;
+    if (wsmem > 48 * 1024 && (e = weights_set_smem_limit(wsmem)) != cudaSuccess) { free(h); return fail_cuda(e); }
+
+    h->grid_dispatch = h->sms * dispatch_blocks_per_sm();
+    h->grid_combine = h->sms * combine_blocks_per_sm(d.K);
+    h->grid_weights = h->sms * weights_blocks_per_sm();
+
+    const size_t wsb = workspace_bytes(d);
+    if ((e = cudaMalloc(&h->ws_mem, wsb)) != cudaSuccess) { free(h); return fail_cuda(e); }
+    if ((e = cudaMemset(h->ws_mem, 0, wsb)) != cudaSuccess) {
+        cudaFree(h->ws_mem);
+        free(h);
+        return fail_cuda(e);
+    }
+    carve_workspace(d, h->ws_mem, &h->ws);
+    *out = h;
+    return MOONEP_OK;
+}
+
+extern "C" int moonep_destroy(moonep_handle_t h) {
+    if (!h) return MOONEP_OK;
+    cudaError_t e = cudaSuccess;
+    if (h->ws_mem) e = cudaFree(h->ws_mem);
+    free(h);
+    return e == cudaSuccess ? MOONEP_OK : MOONEP_ERR_CUDA;
+}
+
+extern "C" int64_t moonep_nvs(moonep_handle_t h) { return h ? (int64_t)h->d.nvs : MOONEP_ERR_NULL; }
+
+extern "C" int moonep_get_config(moonep_handle_t h, moonep_config_t *out) {
+    if (!h || !out) return MOONEP_ERR_NULL;
+    *out = h->cfg;
+    return MOONEP_OK;
+}
+
+extern "C" int moonep_plan(moonep_handle_t h, const int32_t *topk, const int32_t *tokens_per_expert,
+                           const moonep_plan_t *plan, moonep_stream_t stream) {
+    if (!h || !topk || !plan_ok(plan)) return MOONEP_ERR_NULL;
+    if (h->d.B > 0 && !plan->slot_expert) return MOONEP_ERR_NULL;
+    PlanArgs a;
+    a.d = h->d;
+    a.topk = topk;
+    a.tpe = tokens_per_expert;
+    a.plan = *plan;
+    a.ws = h->ws;
+    const cudaError_t e = launch_plan(a, h->sms, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MOONEP_OK : fail_cuda(e);
+}
+
+static CopyArgs copy_args(moonep_handle_t h, const moonep_plan_t *plan) {
+    CopyArgs a;
+    a.d = h->d;
+    a.dst = plan->dst;
+    a.status = plan->status;
+    a.status_rw = plan->status;
+    return a;
+}
+
+extern "C" int moonep_dispatch(moonep_handle_t h, const moonep_plan_t *plan, const void *hidden,
+                               const float *route_weights, void *hidden_nvs, float *route_weights_nvs,
+                               moonep_stream_t stream) {
+    if (!h || !plan || !plan->dst || !plan->status || !hidden || !hidden_nvs) return MOONEP_ERR_NULL;
+    if (!aligned16(hidden) || !aligned16(hidden_nvs)) return MOONEP_ERR_ALIGN;
+    CopyArgs a = copy_args(h, plan);
+    a.src = hidden;
+    a.w = route_weights;
+    a.out = hidden_nvs;
+    a.w_out = route_weights_nvs;
+    const cudaError_t e = launch_dispatch(a, h->grid_dispatch, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MOONEP_OK : fail_cuda(e);
+}
+
+extern "C" int moonep_combine(moonep_handle_t h, const moonep_plan_t *plan, const void *hidden_nvs,
+                              const float *route_weights_nvs, void *out, float *gathered_weights,
+                              moonep_stream_t stream) {
+    if (!h || !plan || !plan->dst || !plan->status || !hidden_nvs || !out) return MOONEP_ERR_NULL;
+    if (!aligned16(hidden_nvs) || !aligned16(out)) return MOONEP_ERR_ALIGN;
+    CopyArgs a = copy_args(h, plan);
+    a.src = hidden_nvs;
+    a.w = route_weights_nvs;
+    a.out = out;
+    a.w_out = route_weights_nvs ? gathered_weights : nullptr;
+    const cudaError_t e = launch_combine(a, h->grid_combine, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MOONEP_OK : fail_cuda(e);
+}
+
+static int weight_args(moonep_handle_t h, const moonep_plan_t *plan, int32_t n_proj, const void *const *src,
+                       void *const *dst, int64_t Hp, WeightArgs *a) {
+    if (!h || !plan || !plan->status || !src || !dst) return MOONEP_ERR_NULL;
+    if (n_proj < 1 || n_proj > MOONEP_MAX_PROJ || Hp < 1) return MOONEP_ERR_SIZE;
+    if (h->d.B > 0 && !plan->slot_expert) return MOONEP_ERR_NULL;
+    memset(a, 0, sizeof(*a));
+    a->d = h->d;
+    a->slot_expert = plan->slot_expert;
+    a->status = plan->status;
+    a->n_proj = n_proj;
+    a->hhp = (int64_t)h->d.H * Hp;
+    for (int p = 0; p < n_proj; ++p) {
+        if (!src[p] || !dst[p]) return MOONEP_ERR_NULL;
+        if (!aligned16(src[p]) || !aligned16(dst[p])) return MOONEP_ERR_ALIGN;
+        a->src[p] = src[p];
+        a->dst[p] = dst[p];
+    }
+    return MOONEP_OK;
+}
+
+extern "C" int moonep_prefetch_weight(moonep_handle_t h, const moonep_plan_t *plan, int32_t n_proj,
+                                      const void *const *weights, void *const *pool, int64_t Hp,
+                                      moonep_stream_t stream) {
+    WeightArgs a;
+    const int rc = weight_args(h, plan, n_proj, weights, pool, Hp, &a);
+    if (rc != MOONEP_OK) return rc;
+    if (h->d.B == 0) return MOONEP_OK;  // no slots: nothing to copy
+    const cudaError_t e = launch_prefetch(a, h->grid_weights, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MOONEP_OK : fail_cuda(e);
+}
+
+extern "C" int moonep_reduce_grad(moonep_handle_t h, const moonep_plan_t *plan, int32_t n_proj,
+                                  float *const *grads, float *const *reduce_buffers, int64_t Hp,
+                                  moonep_stream_t stream) {
+    WeightArgs a;
+    // the reduce buffers are the source (read, then zeroed), the grads the destination
+    const int rc = weight_args(h, plan, n_proj, reinterpret_cast<const void *const *>(reduce_buffers),
+                               reinterpret_cast<void *const *>(grads), Hp, &a);
+    if (rc != MOONEP_OK) return rc;
+    if (h->d.B == 0) return MOONEP_OK;
+    const cudaError_t e = launch_reduce_grad(a, h->grid_weights, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MOONEP_OK : fail_cuda(e);
+}
+
+extern "C" int moonep_read_status(const moonep_plan_t *plan, int32_t *status, moonep_stream_t stream) {
+    if (!plan || !plan->status || !status) return MOONEP_ERR_NULL;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(status, plan->status, sizeof(int32_t), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    return e == cudaSuccess ? MOONEP_OK : fail_cuda(e);
+}

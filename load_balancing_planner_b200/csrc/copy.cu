@@ -1,0 +1,226 @@
+// Fused-permute dispatch and combine (MoonEP README, "dispatch fwd",
+// "combine fwd", "dispatch bwd", "combine bwd"; MarkTechPost, "Core idea:
+// dynamic redundant experts", property 3: tokens are written straight into
+// their expert-grouped positions and the buffer views go to the compute).
+//
+// Both kernels are HBM-bound gathers/scatters of whole bf16 rows.  One warp
+// owns one token: lane k (< K) holds the token's k-th destination slot, and
+// the row moves as 16-byte vectors, U vectors per lane in flight, with
+// streaming cache hints (every byte is touched once).  The grid is a whole
+// number of waves over the SMs and walks the tokens in a grid-stride loop.
+#include "moonep_internal.cuh"
+
+namespace moonep {
+
+__device__ __forceinline__ uint4 ld_stream(const uint4 *p) { return __ldcs(p); }
+__device__ __forceinline__ void st_stream(uint4 *p, const uint4 &v) { __stcs(p, v); }
+
+// ---- dispatch ----------------------------------------------------------------
+template <int U>
+__global__ void __launch_bounds__(256) dispatch_kernel(CopyArgs a) {
+    pdl_wait();
+    if (*a.status != 0) return;
+    const Dims &d = a.d;
+    const int lane = threadIdx.x & 31;
+    const int HV = d.H >> 3;
+    const int64_t ntok = (int64_t)d.R * d.S;
+    const int64_t nslots = (int64_t)d.R * d.nvs;
+    const uint4 *src = static_cast<const uint4 *>(a.src);
+    uint4 *buf = static_cast<uint4 *>(a.out);
+    const int64_t wstride = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t tok = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; tok < ntok; tok += wstride) {
+        int dk = -1;
+        if (lane < d.K) {
+            dk = a.dst[tok * d.K + lane];
+            if (dk < 0 || dk >= nslots) {
+                atomicOr(a.status_rw, MOONEP_STATUS_BAD_PLAN);
+                dk = -1;
+            } else if (a.w != nullptr && a.w_out != nullptr) {
+                a.w_out[dk] = __ldcs(a.w + tok * d.K + lane);
+            }
+        }
+        const uint4 *row = src + tok * HV;
+        for (int v0 = 0; v0 < HV; v0 += 32 * U) {
+            uint4 x[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int v = v0 + u * 32 + lane;
+                if (v < HV) x[u] = ld_stream(row + v);
+            }
+            for (int k = 0; k < d.K; ++k) {
+                const int dd = __shfl_sync(0xffffffffu, dk, k);
+                if (dd < 0) continue;
+                uint4 *o = buf + (int64_t)dd * HV;
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int v = v0 + u * 32 + lane;
+                    if (v < HV) st_stream(o + v, x[u]);
+                }
+            }
+        }
+    }
+}
+
+// ---- combine -----------------------------------------------------------------
+__device__ __forceinline__ void fma_bf16x8(float (&acc)[8], const uint4 &y, float w) {
+    const uint32_t q[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        acc[2 * i] = fmaf(w, __uint_as_float(q[i] << 16), acc[2 * i]);
+        acc[2 * i + 1] = fmaf(w, __uint_as_float(q[i] & 0xffff0000u), acc[2 * i + 1]);
+    }
+}
+
+__device__ __forceinline__ uint4 pack_bf16x8(const float (&acc)[8]) {
+    uint32_t q[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+        q[i] = *reinterpret_cast<const uint32_t *>(&h);
+    }
+    return make_uint4(q[0], q[1], q[2], q[3]);
+}
+
+// KT > 0: K known at compile time (all K*U loads of a step in flight);
+// KT == 0: any K, loads issued in groups of 4 rows.
+template <int KT, int U>
+__global__ void __launch_bounds__(256) combine_kernel(CopyArgs a) {
+    pdl_wait();
+    if (*a.status != 0) return;
+    const Dims &d = a.d;
+    const int K = KT > 0 ? KT : d.K;
+    const int lane = threadIdx.x & 31;
+    const int HV = d.H >> 3;
+    const int64_t ntok = (int64_t)d.R * d.S;
+    const int64_t nslots = (int64_t)d.R * d.nvs;
+    const uint4 *y = static_cast<const uint4 *>(a.src);
+    uint4 *out = static_cast<uint4 *>(a.out);
+    const int64_t wstride = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t tok = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; tok < ntok; tok += wstride) {
+        int dk = 0;
+        float wk = 1.0f;
+        if (lane < K) {
+            dk = a.dst[tok * K + lane];
+            if (dk < 0 || dk >= nslots) {
+                atomicOr(a.status_rw, MOONEP_STATUS_BAD_PLAN);
+                dk = 0;
+                wk = 0.0f;
+            } else if (a.w != nullptr) {
+                wk = a.w[dk];
+                if (a.w_out != nullptr) a.w_out[tok * K + lane] = wk;
+            }
+        }
+        uint4 *orow = out + tok * HV;
+        for (int v0 = 0; v0 < HV; v0 += 32 * U) {
+            float acc[U][8];
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[u][i] = 0.0f;
+            if constexpr (KT > 0) {
+                uint4 yv[KT][U];
+#pragma unroll
+                for (int k = 0; k < KT; ++k) {
+                    const int dd = __shfl_sync(0xffffffffu, dk, k);
+                    const uint4 *yrow = y + (int64_t)dd * HV;
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        const int v = v0 + u * 32 + lane;
+                        yv[k][u] = v < HV ? ld_stream(yrow + v) : make_uint4(0, 0, 0, 0);
+                    }
+                }
+#pragma unroll
+                for (int k = 0; k < KT; ++k) {
+                    const float ww = __shfl_sync(0xffffffffu, wk, k);
+#pragma unroll
+                    for (int u = 0; u < U; ++u) fma_bf16x8(acc[u], yv[k][u], ww);
+                }
+            } else {
+                for (int k0 = 0; k0 < K; k0 += 4) {
+                    uint4 yv[4][U];
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const int dd = __shfl_sync(0xffffffffu, dk, (k0 + kk) & 31);
+                        const uint4 *yrow = y + (int64_t)dd * HV;
+#pragma unroll
+                        for (int u = 0; u < U; ++u) {
+                            const int v = v0 + u * 32 + lane;
+                            yv[kk][u] = (v < HV && k0 + kk < K) ? ld_stream(yrow + v) : make_uint4(0, 0, 0, 0);
+                        }
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const float ww = __shfl_sync(0xffffffffu, wk, (k0 + kk) & 31);
+                        if (k0 + kk < K) {
+#pragma unroll
+                            for (int u = 0; u < U; ++u) fma_bf16x8(acc[u], yv[kk][u], ww);
+                        }
+                    }
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int v = v0 + u * 32 + lane;
+                if (v < HV) st_stream(orow + v, pack_bf16x8(acc[u]));
+            }
+        }
+    }
+}
+
+// ---- launch ------------------------------------------------------------------
+static cudaLaunchAttribute pdl_attr() {
+    cudaLaunchAttribute at;
+    at.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at.val.programmaticStreamSerializationAllowed = 1;
+    return at;
+}
+
+template <typename Kern>
+static cudaError_t launch_pdl(Kern kern, int grid, cudaStream_t st, const CopyArgs &a) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(256);
+    cfg.stream = st;
+    cudaLaunchAttribute at[1] = {pdl_attr()};
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+constexpr int kDispatchU = 4;
+
+cudaError_t launch_dispatch(const CopyArgs &a, int grid, cudaStream_t st) {
+    return launch_pdl(dispatch_kernel<kDispatchU>, grid, st, a);
+}
+
+int dispatch_blocks_per_sm() {
+    int n = 0;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, dispatch_kernel<kDispatchU>, 256, 0);
+    return n > 0 ? n : 1;
+}
+
+cudaError_t launch_combine(const CopyArgs &a, int grid, cudaStream_t st) {
+    switch (a.d.K) {
+        case 1: return launch_pdl(combine_kernel<1, 4>, grid, st, a);
+        case 2: return launch_pdl(combine_kernel<2, 4>, grid, st, a);
+        case 4: return launch_pdl(combine_kernel<4, 2>, grid, st, a);
+        case 6: return launch_pdl(combine_kernel<6, 2>, grid, st, a);
+        case 8: return launch_pdl(combine_kernel<8, 2>, grid, st, a);
+        default: return launch_pdl(combine_kernel<0, 2>, grid, st, a);
+    }
+}
+
+int combine_blocks_per_sm(int K) {
+    int n = 0;
+    switch (K) {
+        case 1: cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, combine_kernel<1, 4>, 256, 0); break;
+        case 2: cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, combine_kernel<2, 4>, 256, 0); break;
+        case 4: cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, combine_kernel<4, 2>, 256, 0); break;
+        case 6: cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, combine_kernel<6, 2>, 256, 0); break;
+        case 8: cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, combine_kernel<8, 2>, 256, 0); break;
+        default: cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, combine_kernel<0, 2>, 256, 0); break;
+    }
+    return n > 0 ? n : 1;
+}
+
+}  // namespace moonep

@@ -1,0 +1,243 @@
+// Weight prefetch and grad-slot reduction (MoonEP README, "Weight buffer",
+// "Grad buffer", "dispatch fwd" prefetch_weight, "dispatch bwd" reduce_grad;
+// MarkTechPost, "Memory contract").
+//
+// Both walk the used prefetch slots of all ranks grouped by expert: the first
+// slot (in (rank, slot) order) that holds an expert leads, and a linked list
+// in shared memory chains the later slots holding the same expert.  Work is
+// cut into (projection, leading slot, tile of the [H, H'] matrix) units taken
+// by a grid-stride loop, so every expert matrix is read once:
+//   prefetch:    load a bf16 tile of W[e], store it to every slot holding e;
+//   reduce_grad: load the fp32 tile of G[e], add every holder's tile in
+//                ascending slot order, store G[e], store zeros to the holders.
+#include "moonep_internal.cuh"
+
+namespace moonep {
+
+constexpr int kWThreads = 256;
+constexpr int kWVec = 4;                          // 16-byte vectors per thread per tile
+constexpr int kWTile = kWThreads * kWVec;         // vectors per tile
+
+// Binary search for expert e in one rank's slot row: used slots first, in
+// ascending expert order, then -1s (the layout moonep_plan writes).
+__device__ __forceinline__ int find_slot(const int32_t *row, int B, int e) {
+    int lo = 0, hi = B;
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        const int v = row[mid];
+        if (v >= 0 && v < e) lo = mid + 1;
+        else hi = mid;
+    }
+    return (lo < B && row[lo] == e) ? lo : -1;
+}
+
+__device__ __forceinline__ int warp_incl_scan_w(int v) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += n;
+    }
+    return v;
+}
+
+// Shared-memory slot tables: se[RB] expert or -1, nxt[RB] next slot holding
+// the same expert (-1 = last), lead[] leading slots in ascending order.
+// Returns the number of leaders, or -1 after flagging a malformed slot table.
+__device__ int build_slot_lists(const WeightArgs &a, int32_t *se, int32_t *nxt, int32_t *lead) {
+    __shared__ int s_bad;
+    __shared__ int s_warp[kWThreads / 32];
+    const int R = a.d.R, B = a.d.B, E = a.d.E, RB = R * B;
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    if (tid == 0) s_bad = 0;
+    __syncthreads();
+    for (int s = tid; s < RB; s += kWThreads) {
+        const int e = a.slot_expert[s];
+        if (e < -1 || e >= E) s_bad = 1;
+        se[s] = e;
+    }
+    __syncthreads();
+    for (int s = tid; s < RB; s += kWThreads) {
+        const int e = se[s];
+        if (s % B != 0 && e >= 0) {
+            const int prev = se[s - 1];
+            if (prev < 0 || prev >= e) s_bad = 1;  // used slots first, ascending, distinct
+        }
+    }
+    __syncthreads();
+    if (s_bad) {
+        if (tid == 0) atomicOr(a.status, MOONEP_STATUS_BAD_PLAN);
+        return -1;
+    }
+    const int per = (RB + kWThreads - 1) / kWThreads;  // <= 16 (RB <= 4096)
+    const int s0 = min(RB, tid * per), s1 = min(RB, s0 + per);
+    unsigned mask = 0;
+    int cnt = 0;
+    for (int s = s0; s < s1; ++s) {
+        const int e = se[s];
+        const int r = s / B;
+        int next = -1;
+        bool leader = e >= 0;
+        if (e >= 0) {
+            for (int r2 = 0; r2 < r && leader; ++r2)
+                if (find_slot(se + r2 * B, B, e) >= 0) leader = false;
+            for (int r2 = r + 1; r2 < R; ++r2) {
+                const int j = find_slot(se + r2 * B, B, e);
+                if (j >= 0) {
+                    next = r2 * B + j;
+                    break;
+                }
+            }
+        }
+        nxt[s] = next;
+        if (leader) {
+            mask |= 1u << (s - s0);
+            ++cnt;
+        }
+    }
+    // leaders in ascending slot order: block-wide exclusive scan of the counts
+    const int incl = warp_incl_scan_w(cnt);
+    if (lane == 31) s_warp[w] = incl;
+    __syncthreads();
+    if (w == 0) {
+        const int x = lane < kWThreads / 32 ? s_warp[lane] : 0;
+        const int xi = warp_incl_scan_w(x);
+        if (lane < kWThreads / 32) s_warp[lane] = xi;
+    }
+    __syncthreads();
+    int pos = (w > 0 ? s_warp[w - 1] : 0) + incl - cnt;
+    const int total = s_warp[kWThreads / 32 - 1];
+    for (int s = s0; s < s1; ++s)
+        if (mask & (1u << (s - s0))) lead[pos++] = s;
+    __syncthreads();
+    return total;
+}
+
+__global__ void __launch_bounds__(kWThreads) prefetch_kernel(WeightArgs a) {
+    pdl_wait();
+    if (*a.status != 0) return;
+    extern __shared__ int32_t wsm[];
+    const int RB = a.d.R * a.d.B;
+    int32_t *se = wsm, *nxt = wsm + RB, *lead = wsm + 2 * RB;
+    const int nlead = build_slot_lists(a, se, nxt, lead);
+    if (nlead <= 0) return;
+    const int64_t nvec = a.hhp / 8;  // bf16: 8 per 16 bytes
+    const int64_t ntiles = (nvec + kWTile - 1) / kWTile;
+    const int64_t units = (int64_t)a.n_proj * nlead * ntiles;
+    for (int64_t u = blockIdx.x; u < units; u += gridDim.x) {
+        const int p = (int)(u / ((int64_t)nlead * ntiles));
+        const int64_t rem = u - (int64_t)p * nlead * ntiles;
+        const int s = lead[rem / ntiles];
+        const int64_t t0 = (rem % ntiles) * kWTile;
+        const uint4 *src = static_cast<const uint4 *>(a.src[p]) + (int64_t)se[s] * nvec + t0;
+        uint4 x[kWVec];
+#pragma unroll
+        for (int i = 0; i < kWVec; ++i) {
+            const int64_t v = t0 + i * kWThreads + threadIdx.x;
+            if (v < nvec) x[i] = __ldcs(src + i * kWThreads + threadIdx.x);
+        }
+        for (int j = s; j >= 0; j = nxt[j]) {
+            uint4 *dst = static_cast<uint4 *>(a.dst[p]) + (int64_t)j * nvec + t0;
+#pragma unroll
+            for (int i = 0; i < kWVec; ++i) {
+                const int64_t v = t0 + i * kWThreads + threadIdx.x;
+                if (v < nvec) __stcs(dst + i * kWThreads + threadIdx.x, x[i]);
+            }
+        }
+    }
+}
+
+// a.src[p] = reduce buffer [R*B, H*Hp] (read, then zeroed), a.dst[p] = grads [E, H*Hp].
+__global__ void __launch_bounds__(kWThreads) reduce_grad_kernel(WeightArgs a) {
+    pdl_wait();
+    if (*a.status != 0) return;
+    extern __shared__ int32_t wsm[];
+    const int RB = a.d.R * a.d.B;
+    int32_t *se = wsm, *nxt = wsm + RB, *lead = wsm + 2 * RB;
+    const int nlead = build_slot_lists(a, se, nxt, lead);
+    if (nlead <= 0) return;
+    const int64_t nvec = a.hhp / 4;  // fp32: 4 per 16 bytes
+    const int64_t ntiles = (nvec + kWTile - 1) / kWTile;
+    const int64_t units = (int64_t)a.n_proj * nlead * ntiles;
+    const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int64_t u = blockIdx.x; u < units; u += gridDim.x) {
+        const int p = (int)(u / ((int64_t)nlead * ntiles));
+        const int64_t rem = u - (int64_t)p * nlead * ntiles;
+        const int s = lead[rem / ntiles];
+        const int64_t t0 = (rem % ntiles) * kWTile;
+        float4 *g = static_cast<float4 *>(a.dst[p]) + (int64_t)se[s] * nvec + t0;
+        float4 *rb = static_cast<float4 *>(const_cast<void *>(a.src[p]));
+        float4 acc[kWVec];
+#pragma unroll
+        for (int i = 0; i < kWVec; ++i) {
+            const int64_t v = t0 + i * kWThreads + threadIdx.x;
+            acc[i] = v < nvec ? __ldcs(g + i * kWThreads + threadIdx.x) : zero;
+        }
+        for (int j = s; j >= 0; j = nxt[j]) {
+            const float4 *slot = rb + (int64_t)j * nvec + t0;
+#pragma unroll
+            for (int i = 0; i < kWVec; ++i) {
+                const int64_t v = t0 + i * kWThreads + threadIdx.x;
+                if (v < nvec) {
+                    const float4 x = __ldcs(slot + i * kWThreads + threadIdx.x);
+                    acc[i].x = __fadd_rn(acc[i].x, x.x);
+                    acc[i].y = __fadd_rn(acc[i].y, x.y);
+                    acc[i].z = __fadd_rn(acc[i].z, x.z);
+                    acc[i].w = __fadd_rn(acc[i].w, x.w);
+                }
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < kWVec; ++i) {
+            const int64_t v = t0 + i * kWThreads + threadIdx.x;
+            if (v < nvec) __stcs(g + i * kWThreads + threadIdx.x, acc[i]);
+        }
+        for (int j = s; j >= 0; j = nxt[j]) {
+            float4 *slot = rb + (int64_t)j * nvec + t0;
+#pragma unroll
+            for (int i = 0; i < kWVec; ++i) {
+                const int64_t v = t0 + i * kWThreads + threadIdx.x;
+                if (v < nvec) __stcs(slot + i * kWThreads + threadIdx.x, zero);
+            }
+        }
+    }
+}
+
+static size_t weights_smem(const WeightArgs &a) { return sizeof(int32_t) * 3 * (size_t)a.d.R * a.d.B; }
+
+template <typename Kern>
+static cudaError_t launch_w(Kern kern, const WeightArgs &a, int grid, cudaStream_t st) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kWThreads);
+    cfg.dynamicSmemBytes = weights_smem(a);
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+cudaError_t launch_prefetch(const WeightArgs &a, int grid, cudaStream_t st) {
+    return launch_w(prefetch_kernel, a, grid, st);
+}
+
+cudaError_t launch_reduce_grad(const WeightArgs &a, int grid, cudaStream_t st) {
+    return launch_w(reduce_grad_kernel, a, grid, st);
+}
+
+int weights_blocks_per_sm() {
+    int n = 0;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, reduce_grad_kernel, kWThreads, 0);
+    return n > 0 ? n : 1;
+}
+
+cudaError_t weights_set_smem_limit(size_t bytes) {
+    cudaError_t e = cudaFuncSetAttribute(prefetch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(reduce_grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+}  // namespace moonep

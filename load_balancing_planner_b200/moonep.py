@@ -1,0 +1,243 @@
+"""Thin Python binding of libmoonep (include/moonep.h): argument marshalling only.
+
+Functions carry the C names.  Tensors are torch CUDA tensors; their data
+pointers and the current CUDA stream are passed straight to the C ABI, and
+every step of the hot path runs in the library's kernels.  There is no CPU
+fallback: if the shared library is missing the import fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoonep.so")
+
+OK, ERR_NULL, ERR_CONFIG, ERR_ALIGN, ERR_CUDA, ERR_SIZE = 0, -1, -2, -3, -4, -5
+STATUS_BAD_EXPERT, STATUS_DUP_EXPERT, STATUS_COUNT_MISMATCH, STATUS_BAD_PLAN = 1, 2, 4, 8
+MAX_R, MAX_E, MAX_K, MAX_PROJ = 64, 4096, 32, 8
+TRAINING, INFERENCE = 0, 1
+
+
+class MoonepError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {error_string(code)} ({code})")
+        self.code = code
+
+
+class Config(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("S", "H", "K", "E", "R", "B", "token_padding", "num_sms", "mode")]
+
+
+class PlanStruct(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("dst", "cu_seqlens", "row_counts", "slot_expert", "counts", "assign", "maxvio", "status")]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m load_balancing_planner_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+    sig = {
+        "moonep_create": ([ctypes.POINTER(Config), ctypes.POINTER(P)], ctypes.c_int),
+        "moonep_destroy": ([P], ctypes.c_int),
+        "moonep_nvs": ([P], i64),
+        "moonep_get_config": ([P, ctypes.POINTER(Config)], ctypes.c_int),
+        "moonep_plan": ([P, P, P, ctypes.POINTER(PlanStruct), P], ctypes.c_int),
+        "moonep_dispatch": ([P, ctypes.POINTER(PlanStruct), P, P, P, P, P], ctypes.c_int),
+        "moonep_combine": ([P, ctypes.POINTER(PlanStruct), P, P, P, P, P], ctypes.c_int),
+        "moonep_prefetch_weight": ([P, ctypes.POINTER(PlanStruct), i32, P, P, i64, P], ctypes.c_int),
+        "moonep_reduce_grad": ([P, ctypes.POINTER(PlanStruct), i32, P, P, i64, P], ctypes.c_int),
+        "moonep_read_status": ([ctypes.POINTER(PlanStruct), ctypes.POINTER(i32), P], ctypes.c_int),
+        "moonep_error_string": ([ctypes.c_int], ctypes.c_char_p),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(L, name)
+        f.argtypes = args
+        f.restype = res
+    return L
+
+
+lib = _load()
+EXPORTS = ("moonep_create", "moonep_destroy", "moonep_nvs", "moonep_get_config", "moonep_plan",
+           "moonep_dispatch", "moonep_combine", "moonep_prefetch_weight", "moonep_reduce_grad",
+           "moonep_read_status", "moonep_error_string")
+
+
+def error_string(code: int) -> str:
+    return lib.moonep_error_string(code).decode()
+
+
+def _check(rc: int, what: str):
+    if rc != OK:
+        raise MoonepError(rc, what)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("moonep takes CUDA tensors")
+    if not t.is_contiguous():
+        raise ValueError("moonep takes contiguous tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _expect(t, shape, dtype, name):
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape) or t.dtype != dtype:
+        raise ValueError(f"{name}: expected {tuple(shape)} {dtype}, got {tuple(t.shape)} {t.dtype}")
+
+
+class Handle:
+    """Owns a moonep_handle_t (and its planning workspace)."""
+
+    def __init__(self, ptr: int, cfg: Config):
+        self.ptr = ctypes.c_void_p(ptr)
+        self.cfg = cfg
+        self.nvs = int(lib.moonep_nvs(self.ptr))
+
+    def __getattr__(self, k):
+        if k in ("S", "H", "K", "E", "R", "B", "token_padding", "num_sms", "mode"):
+            return getattr(self.cfg, k)
+        raise AttributeError(k)
+
+    def close(self):
+        if self.ptr:
+            _check(lib.moonep_destroy(self.ptr), "moonep_destroy")
+            self.ptr = ctypes.c_void_p(0)
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class Plan:
+    """Device arrays of one plan (caller-owned, see moonep_plan_t)."""
+
+    def __init__(self, h: Handle, device=None):
+        dev = device or torch.device("cuda", torch.cuda.current_device())
+        R, S, K, E, B = h.R, h.S, h.K, h.E, h.B
+        i32 = dict(dtype=torch.int32, device=dev)
+        self.dst = torch.empty((R, S, K), **i32)
+        self.cu_seqlens = torch.empty((R, E + B), **i32)
+        self.row_counts = torch.empty((R, E + B), **i32)
+        self.slot_expert = torch.empty((R, max(B, 1)), **i32)
+        self.counts = torch.empty((R, E), **i32)
+        self.assign = torch.empty((R, 4), **i32)
+        self.maxvio = torch.empty((1,), dtype=torch.float32, device=dev)
+        self.status = torch.zeros((1,), **i32)
+        self.struct = PlanStruct(*(t.data_ptr() for t in (
+            self.dst, self.cu_seqlens, self.row_counts, self.slot_expert, self.counts,
+            self.assign, self.maxvio, self.status)))
+        self.nvs = h.nvs
+        self.B = B
+
+    def slots(self):
+        return self.slot_expert[:, : self.B]
+
+
+def moonep_create(S, H, K, E, R, B=None, token_padding=128, num_sms=0, mode=TRAINING) -> Handle:
+    B = E // R if B is None else B
+    cfg = Config(S, H, K, E, R, B, token_padding, num_sms, mode)
+    out = ctypes.c_void_p()
+    _check(lib.moonep_create(ctypes.byref(cfg), ctypes.byref(out)), "moonep_create")
+    return Handle(out.value, cfg)
+
+
+def moonep_destroy(h: Handle):
+    h.close()
+
+
+def moonep_nvs(h: Handle) -> int:
+    return int(lib.moonep_nvs(h.ptr))
+
+
+def moonep_plan(h: Handle, topk, tokens_per_expert=None, plan: Plan | None = None, stream=None) -> Plan:
+    _expect(topk, (h.R, h.S, h.K), torch.int32, "topk")
+    _expect(tokens_per_expert, (h.R, h.E), torch.int32, "tokens_per_expert")
+    plan = plan or Plan(h, topk.device)
+    _check(lib.moonep_plan(h.ptr, _ptr(topk), _ptr(tokens_per_expert), ctypes.byref(plan.struct),
+                           _stream(stream)), "moonep_plan")
+    return plan
+
+
+def moonep_dispatch(h: Handle, plan: Plan, hidden, route_weights=None, hidden_nvs=None,
+                    route_weights_nvs=None, stream=None):
+    _expect(hidden, (h.R, h.S, h.H), torch.bfloat16, "hidden")
+    _expect(route_weights, (h.R, h.S, h.K), torch.float32, "route_weights")
+    if hidden_nvs is None:
+        hidden_nvs = torch.empty((h.R, h.nvs, h.H), dtype=torch.bfloat16, device=hidden.device)
+    if route_weights is not None and route_weights_nvs is None:
+        route_weights_nvs = torch.empty((h.R, h.nvs), dtype=torch.float32, device=hidden.device)
+    _expect(hidden_nvs, (h.R, h.nvs, h.H), torch.bfloat16, "hidden_nvs")
+    _expect(route_weights_nvs, (h.R, h.nvs), torch.float32, "route_weights_nvs")
+    _check(lib.moonep_dispatch(h.ptr, ctypes.byref(plan.struct), _ptr(hidden), _ptr(route_weights),
+                               _ptr(hidden_nvs), _ptr(route_weights_nvs), _stream(stream)), "moonep_dispatch")
+    return hidden_nvs, route_weights_nvs
+
+
+def moonep_combine(h: Handle, plan: Plan, hidden_nvs, route_weights_nvs=None, out=None,
+                   gathered_weights=None, gather=True, stream=None):
+    _expect(hidden_nvs, (h.R, h.nvs, h.H), torch.bfloat16, "hidden_nvs")
+    _expect(route_weights_nvs, (h.R, h.nvs), torch.float32, "route_weights_nvs")
+    if out is None:
+        out = torch.empty((h.R, h.S, h.H), dtype=torch.bfloat16, device=hidden_nvs.device)
+    if gather and route_weights_nvs is not None and gathered_weights is None:
+        gathered_weights = torch.empty((h.R, h.S, h.K), dtype=torch.float32, device=hidden_nvs.device)
+    _expect(out, (h.R, h.S, h.H), torch.bfloat16, "out")
+    _expect(gathered_weights, (h.R, h.S, h.K), torch.float32, "gathered_weights")
+    _check(lib.moonep_combine(h.ptr, ctypes.byref(plan.struct), _ptr(hidden_nvs), _ptr(route_weights_nvs),
+                              _ptr(out), _ptr(gathered_weights), _stream(stream)), "moonep_combine")
+    return out, gathered_weights
+
+
+def _ptr_array(ts):
+    arr = (ctypes.c_void_p * len(ts))(*[t.data_ptr() for t in ts])
+    for t in ts:
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("moonep takes contiguous CUDA tensors")
+    return arr
+
+
+def moonep_prefetch_weight(h: Handle, plan: Plan, weights, pool, stream=None):
+    """weights: list of [E, H, Hp] bf16; pool: list of [R, B, H, Hp] bf16."""
+    if len(weights) != len(pool) or not weights:
+        raise ValueError("one pool per weight tensor")
+    Hp = weights[0].shape[-1]
+    for W, P in zip(weights, pool):
+        _expect(W, (h.E, h.H, Hp), torch.bfloat16, "weights")
+        _expect(P, (h.R, h.B, h.H, Hp), torch.bfloat16, "pool")
+    _check(lib.moonep_prefetch_weight(h.ptr, ctypes.byref(plan.struct), len(weights), _ptr_array(weights),
+                                      _ptr_array(pool), Hp, _stream(stream)), "moonep_prefetch_weight")
+
+
+def moonep_reduce_grad(h: Handle, plan: Plan, grads, reduce_buffers, stream=None):
+    """grads: list of [E, H, Hp] fp32; reduce_buffers: list of [R, B, H, Hp] fp32."""
+    if len(grads) != len(reduce_buffers) or not grads:
+        raise ValueError("one reduce buffer per grad tensor")
+    Hp = grads[0].shape[-1]
+    for G, RB in zip(grads, reduce_buffers):
+        _expect(G, (h.E, h.H, Hp), torch.float32, "grads")
+        _expect(RB, (h.R, h.B, h.H, Hp), torch.float32, "reduce_buffers")
+    _check(lib.moonep_reduce_grad(h.ptr, ctypes.byref(plan.struct), len(grads), _ptr_array(grads),
+                                  _ptr_array(reduce_buffers), Hp, _stream(stream)), "moonep_reduce_grad")
+
+
+def moonep_read_status(plan: Plan, stream=None) -> int:
+    st = ctypes.c_int32(0)
+    _check(lib.moonep_read_status(ctypes.byref(plan.struct), ctypes.byref(st), _stream(stream)),
+           "moonep_read_status")
+    return int(st.value)

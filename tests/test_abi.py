@@ -1,0 +1,79 @@
+"""The C ABI library loads and exports every symbol include/moonep.h declares;
+host-side validation rejects bad configurations before touching the GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from tests.conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "moonep.h")
+
+
+def declared_symbols():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"MOONEP_API\s+[\w\s\*]*?\b(moonep_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_hot_path():
+    names = declared_symbols()
+    for n in ("moonep_plan", "moonep_dispatch", "moonep_combine", "moonep_prefetch_weight",
+              "moonep_reduce_grad", "moonep_create", "moonep_destroy"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    from load_balancing_planner_b200 import build
+    path = build.build()
+    lib = ctypes.CDLL(path)
+    for n in declared_symbols():
+        assert hasattr(lib, n), f"{n} declared but not exported"
+
+
+def test_binding_covers_every_declared_symbol():
+    from load_balancing_planner_b200 import moonep
+    assert set(declared_symbols()) == set(moonep.EXPORTS)
+
+
+def test_error_strings():
+    from load_balancing_planner_b200 import moonep
+    assert moonep.error_string(moonep.ERR_CONFIG) == "configuration rejected"
+    assert moonep.error_string(0) == "ok"
+
+
+@pytest.mark.parametrize("bad", [
+    dict(E=10, R=4),             # E % R != 0
+    dict(K=9, E=8),              # K > E
+    dict(H=100),                 # H % 8 != 0
+    dict(B=1, mode=0),           # training needs B >= E/R
+    dict(R=65, E=65 * 4),        # R past the limit
+    dict(E=8192, R=8),           # E past the limit
+    dict(K=33, E=64),            # K past the limit
+    dict(token_padding=0),
+    dict(mode=2),
+    dict(S=0),
+    dict(S=1 << 20, K=32, R=64, E=256),  # R*S*K >= 2^31
+])
+def test_create_rejects_bad_configs_without_a_gpu(bad):
+    from load_balancing_planner_b200 import moonep
+    cfg = dict(S=64, H=128, K=2, E=8, R=2, B=4, token_padding=8, num_sms=0, mode=0)
+    cfg.update(bad)
+    c = moonep.Config(*(cfg[k] for k in ("S", "H", "K", "E", "R", "B", "token_padding", "num_sms", "mode")))
+    out = ctypes.c_void_p(123)
+    rc = moonep.lib.moonep_create(ctypes.byref(c), ctypes.byref(out))
+    assert rc == moonep.ERR_CONFIG
+    assert out.value is None
+
+
+def test_null_arguments_are_rejected():
+    from load_balancing_planner_b200 import moonep
+    P = ctypes.c_void_p
+    assert moonep.lib.moonep_create(None, ctypes.byref(P())) == moonep.ERR_NULL
+    assert moonep.lib.moonep_plan(None, None, None, None, None) == moonep.ERR_NULL
+    assert moonep.lib.moonep_dispatch(None, None, None, None, None, None, None) == moonep.ERR_NULL
+    assert moonep.lib.moonep_combine(None, None, None, None, None, None, None) == moonep.ERR_NULL
+    assert moonep.lib.moonep_prefetch_weight(None, None, 1, None, None, 8, None) == moonep.ERR_NULL
+    assert moonep.lib.moonep_reduce_grad(None, None, 1, None, None, 8, None) == moonep.ERR_NULL
+    assert moonep.lib.moonep_destroy(None) == moonep.OK
+    assert moonep.lib.moonep_nvs(None) < 0

@@ -221,7 +221,8 @@ def test_roundtrip_unweighted_is_K_times_x():
         xb = synth.bf16_bits(x)
         buf, _ = oracle.dispatch(p["dst"], xb, None, p["nvs"])
         out, _ = oracle.combine(p["dst"], buf, None)
-        want = (x.to(torch.float32) * K).to(torch.bfloat16)
+        # the sum starts from +0, so x = -0 gives +0 (adding 0.0 does the same)
+        want = (x.to(torch.float32) * K + 0.0).to(torch.bfloat16)
         assert np.array_equal(out, synth.bf16_bits(want))
 
 
@@ -231,7 +232,7 @@ def test_roundtrip_softmax_weights_is_identity():
     xb = synth.bf16_bits(x)
     buf, w_nvs = oracle.dispatch(p["dst"], xb, w, p["nvs"])
     out, gw = oracle.combine(p["dst"], buf, w_nvs)
-    assert np.array_equal(out, xb)
+    assert np.array_equal(out, synth.bf16_bits((x.to(torch.float32) + 0.0).to(torch.bfloat16)))
     assert np.array_equal(gw, w)
 
 

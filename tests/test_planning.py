@@ -1,0 +1,97 @@
+"""GPU planner == oracle planner, bit for bit: dst, cu_seqlens, row_counts,
+slot_expert, counts, assign, maxvio, status; plus the page invariants checked
+independently on the GPU plan."""
+import numpy as np
+import pytest
+
+import oracle
+from tests.gpu_util import assert_plans_equal, gpu_plan, plan_to_numpy, problem
+from tests.plan_checks import check_plan
+
+pytestmark = pytest.mark.gpu
+
+# (name, R, S, K, E, B, token_padding, mode, routing profile, maxvio sweep)
+CASES = [
+    ("tiny", 2, 64, 2, 8, 4, 8, 0, "boost0", [1.0]),
+    ("zipf", 8, 1024, 8, 64, 8, 128, 0, "zipf", [0.0, 0.5, 1.0, 2.0]),
+    ("train", 8, 4096, 8, 256, 32, 128, 0, "hot8", [0.0, 0.5, 1.0, 2.0, 4.0]),
+    ("infer", 8, 4096, 8, 256, 4, 128, 1, "hot8", [1.0, 4.0]),
+    ("ragged", 3, 1000, 3, 24, 8, 16, 0, "hot8", [1.5]),
+    ("one_rank", 1, 700, 4, 16, 16, 8, 0, "zipf", [2.0]),
+    ("k1_tp1", 8, 64, 1, 8, 1, 1, 0, "boost0", [3.0]),
+    ("no_slots", 4, 333, 3, 24, 0, 16, 1, "hot8", [1.5]),
+    ("wide_e", 4, 600, 8, 1024, 256, 64, 0, "hot8", [2.0]),
+    ("max_e", 8, 300, 8, 4096, 512, 16, 0, "hot8", [2.0]),
+    ("k32", 2, 100, 32, 64, 32, 4, 0, "zipf", [0.5]),
+    ("many_ranks", 64, 40, 4, 256, 4, 8, 0, "hot8", [3.0]),
+]
+
+
+def _ids():
+    out = []
+    for c in CASES:
+        for mv in c[9]:
+            out.append(pytest.param(c, mv, id=f"{c[0]}-mv{mv}"))
+    return out
+
+
+@pytest.mark.parametrize("case,mv", _ids())
+def test_plan_matches_oracle(cuda, case, mv):
+    from load_balancing_planner_b200 import moonep
+    name, R, S, K, E, B, tp, mode, profile, _ = case
+    tk, tpe, _ = problem(R, S, K, E, mv, profile, seed=11)
+    want = oracle.plan(tk, E, B, tp, mode, tpe)
+    assert want["status"] == 0
+    h = moonep.moonep_create(S, 8, K, E, R, B, tp, mode=mode)
+    got = plan_to_numpy(gpu_plan(h, tk, tpe))
+    assert_plans_equal(got, want)
+    check_plan(tk, got, E, B, tp, mode)
+    h.close()
+
+
+def test_handle_reuse_leaves_no_state(cuda):
+    # plan A, plan B, plan A again on one handle: the workspace is reset by
+    # every call, so the third plan equals the first
+    from load_balancing_planner_b200 import moonep
+    R, S, K, E, B, tp = 8, 1024, 8, 64, 8, 128
+    tka, tpea, _ = problem(R, S, K, E, 2.0, "zipf", seed=1)
+    tkb, tpeb, _ = problem(R, S, K, E, 0.5, "zipf", seed=2)
+    h = moonep.moonep_create(S, 8, K, E, R, B, tp)
+    a1 = plan_to_numpy(gpu_plan(h, tka, tpea))
+    b = plan_to_numpy(gpu_plan(h, tkb, tpeb))
+    a2 = plan_to_numpy(gpu_plan(h, tka, tpea))
+    assert_plans_equal(a1, oracle.plan(tka, E, B, tp, 0, tpea))
+    assert_plans_equal(b, oracle.plan(tkb, E, B, tp, 0, tpeb))
+    assert_plans_equal(a2, a1)
+    h.close()
+
+
+def test_plan_without_local_counts(cuda):
+    from load_balancing_planner_b200 import moonep
+    R, S, K, E, B, tp = 8, 1024, 8, 64, 8, 128
+    tk, _, _ = problem(R, S, K, E, 1.0, "zipf", seed=4)
+    h = moonep.moonep_create(S, 8, K, E, R, B, tp)
+    assert_plans_equal(plan_to_numpy(gpu_plan(h, tk, None)), oracle.plan(tk, E, B, tp, 0))
+    h.close()
+
+
+def test_golden_plans_on_gpu(cuda):
+    import json
+    import os
+    from load_balancing_planner_b200 import moonep
+    gdir = os.path.join(os.path.dirname(__file__), "golden")
+    for f in sorted(os.listdir(gdir)):
+        if not f.startswith("plan_"):
+            continue
+        g = json.load(open(os.path.join(gdir, f)))
+        c = g["config"]
+        tk = np.array(g["topk"], np.int32)
+        R, S, K = tk.shape
+        h = moonep.moonep_create(S, 8, K, c["E"], R, c["B"], c["tp"], mode=c["mode"])
+        got = plan_to_numpy(gpu_plan(h, tk))
+        for key, want in g["expect"].items():
+            if isinstance(want, float):
+                assert abs(got[key] - want) < 1e-6, (f, key)
+            else:
+                assert np.array_equal(np.asarray(got[key]), np.asarray(want)), (f, key, np.asarray(got[key]).tolist())
+        h.close()
