@@ -1,0 +1,531 @@
+#!/usr/bin/env python
+"""Benchmark of the balanced expert-parallel hot path on B200.
+
+One step is one MoE layer's forward pass through the library's C ABI at the
+training shape (R=8 emulated EP ranks, S=4096 tokens per rank, K=8, E=256,
+B=32, H=7168, token_padding=128): plan -> dispatch -> combine, with the
+dispatch buffer itself as the expert output.  Steps cycle through routings at
+maxvio 0, 0.5, 1, 2 and 4.  The headline value is dispatch+combine algorithmic
+HBM bytes / wall time of the whole step (planner included).
+
+Also measured in the same run (unless switched off):
+  * per-kernel CUDA-event times (planner us/layer, dispatch and combine GB/s,
+    per-maxvio spread) and the roofline of the dominant kernel;
+  * legs: prefetch_weight at the inference shape (B=4, H'=2048, 3
+    projections) and reduce_grad at the backward shape (B=32, H'=2048 fp32);
+  * e2e: the same step from pinned host buffers, host<->device copies
+    included;
+  * cpu_baseline: the CPU oracle on a bounded sample, one host core.
+
+`--impl reference` times the CPU oracle itself on the same workload (see the
+reference-arm section below).  Multi-GPU (`torchrun ... --gpus N`): every rank
+runs its own independent EP group (weak scaling, no data-path collective);
+time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from load_balancing_planner_b200 import synth  # noqa: E402
+
+METRIC = "dispatch+combine HBM GB/s (% of peak) vs maxvio; planner µs/layer; 1 B200"
+NOMINAL_HBM_GBS = 8000.0
+
+WORKLOADS = {
+    "train": dict(R=8, S=4096, K=8, E=256, B=32, H=7168, tp=128, mode=0, profile="hot8",
+                  maxvio=(0.0, 0.5, 1.0, 2.0, 4.0)),
+    "zipf": dict(R=8, S=1024, K=8, E=64, B=8, H=2048, tp=128, mode=0, profile="zipf",
+                 maxvio=(0.0, 0.5, 1.0, 2.0)),
+    # training rows (H=7168) with fewer tokens: ~1.5 GB on the device, for
+    # profiler captures that must stay small
+    "train_s512": dict(R=8, S=512, K=8, E=256, B=32, H=7168, tp=128, mode=0, profile="hot8",
+                       maxvio=(0.0, 2.0)),
+}
+
+
+def describe(w):
+    return (f"R={w['R']} S={w['S']} K={w['K']} E={w['E']} B={w['B']} H={w['H']} "
+            f"token_padding={w['tp']} {'training' if w['mode'] == 0 else 'inference'}, "
+            f"routing {w['profile']} at maxvio " + "/".join(f"{m:g}" for m in w["maxvio"]))
+
+
+def dc_bytes(R, S, K, H):
+    """Algorithmic bytes of dispatch + combine for one layer (all R ranks):
+    dispatch reads each row once and writes it K times, plus dst, w and w_nvs;
+    combine reads K rows per token and writes one, plus dst and the weights."""
+    disp = R * (S * H * 2 + S * K * H * 2 + 3 * S * K * 4)
+    comb = R * (S * K * H * 2 + S * H * 2 + 2 * S * K * 4)
+    return disp, comb
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+class Clocks:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        self.t0 = time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- helpers
+def setup_dist(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    import torch
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(x, world):
+    import torch
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def make_inputs(w, seed, dev):
+    import torch
+    R, S, K, E, H = w["R"], w["S"], w["K"], w["E"], w["H"]
+    hidden = synth.hidden_bf16(R, S, H, seed).to(dev)
+    weights = torch.from_numpy(synth.route_weights(R, S, K, seed)).to(dev)
+    routes = []
+    for mv in w["maxvio"]:
+        tk, real, _ = synth.routing(R, S, K, E, mv, w["profile"], seed=seed)
+        routes.append(dict(target=mv, realised=real,
+                           topk=torch.from_numpy(tk).to(dev),
+                           tpe=torch.from_numpy(synth.local_counts(tk, E)).to(dev),
+                           topk_np=tk))
+    return hidden, weights, routes
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args, world, rank, local):
+    import torch
+    from load_balancing_planner_b200 import moonep
+
+    w = WORKLOADS[args.config]
+    R, S, K, E, B, H, tp = w["R"], w["S"], w["K"], w["E"], w["B"], w["H"], w["tp"]
+    dev = torch.device("cuda", local if world > 1 else 0)
+    seed = args.seed + rank
+    hidden, weights, routes = make_inputs(w, seed, dev)
+    h = moonep.moonep_create(S, H, K, E, R, B, tp, mode=w["mode"])
+    nvs = h.nvs
+    plan = moonep.Plan(h, dev)
+    buf = torch.empty((R, nvs, H), dtype=torch.bfloat16, device=dev)
+    wn = torch.empty((R, nvs), dtype=torch.float32, device=dev)
+    out = torch.empty((R, S, H), dtype=torch.bfloat16, device=dev)
+    gw = torch.empty((R, S, K), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    npts = len(routes)
+
+    def step(i, ev=None):
+        r = routes[i % npts]
+        if ev:
+            ev[0].record(stream)
+        moonep.moonep_plan(h, r["topk"], r["tpe"], plan)
+        if ev:
+            ev[1].record(stream)
+        moonep.moonep_dispatch(h, plan, hidden, weights, buf, wn)
+        if ev:
+            ev[2].record(stream)
+        moonep.moonep_combine(h, plan, buf, wn, out, gw)
+        if ev:
+            ev[3].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    st = moonep.moonep_read_status(plan)
+    if st != 0:
+        raise RuntimeError(f"plan status {st}")
+
+    clocks = Clocks(local if world > 1 else 0)
+    clocks.start()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    barrier(world)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(i, evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    total_ms = t_start.elapsed_time(t_end)
+    total_ms_max = max_over_ranks(total_ms, world)
+
+    plan_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    disp_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    comb_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    db, cb = dc_bytes(R, S, K, H)
+    peak, peak_kind = peaks()
+    value = world * (db + cb) * args.steps / (total_ms_max * 1e-3) / 1e9
+
+    sweep = {}
+    for j, r in enumerate(routes):
+        idx = [i for i in range(args.steps) if i % npts == j]
+        if not idx:
+            continue
+        dc = statistics.median([disp_ms[i] + comb_ms[i] for i in idx])
+        gbs = (db + cb) / (dc * 1e-3) / 1e9
+        sweep[f"{r['target']:g}"] = dict(
+            realised_maxvio=round(r["realised"], 4), planner_us=round(statistics.median([plan_ms[i] for i in idx]) * 1e3, 2),
+            dispatch_us=round(statistics.median([disp_ms[i] for i in idx]) * 1e3, 1),
+            combine_us=round(statistics.median([comb_ms[i] for i in idx]) * 1e3, 1),
+            dc_gbs=round(gbs, 1), dc_frac_measured=round(gbs / peak, 4), dc_frac_8tbs=round(gbs / NOMINAL_HBM_GBS, 4))
+    dcs = [v["dispatch_us"] + v["combine_us"] for v in sweep.values()]
+    spread = (max(dcs) - min(dcs)) / min(dcs) if dcs else None
+
+    d_avg = statistics.mean(disp_ms)
+    c_avg = statistics.mean(comb_ms)
+    dom = ("dispatch", d_avg, db) if d_avg >= c_avg else ("combine", c_avg, cb)
+    achieved = dom[2] / (dom[1] * 1e-3) / 1e9
+    roofline = dict(bound="hbm", kernel=dom[0], achieved=round(achieved, 1), peak=peak, unit="GB/s",
+                    frac=round(achieved / peak, 4), peak_kind=peak_kind,
+                    frac_of_nominal_8tbs=round(achieved / NOMINAL_HBM_GBS, 4),
+                    traffic=args.traffic, bytes_per_launch=dom[2])
+
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms_max / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": f"{args.config}: " + describe(w), "maxvio": list(w["maxvio"]),
+                   "parallelism": f"EP={R} emulated on each GPU; independent EP groups per GPU",
+                   "l2": "inputs larger than L2 (hidden rows 470 MB, dispatch buffer 4.7 GB per layer)"
+                   if args.config == "train" else "inputs larger than L2",
+                   "step": "plan + dispatch + combine of one layer; combine reads the dispatch buffer"},
+        "planner_us": round(statistics.median(plan_ms) * 1e3, 2),
+        "dispatch_gbs": round(db / (statistics.median(disp_ms) * 1e-3) / 1e9, 1),
+        "combine_gbs": round(cb / (statistics.median(comb_ms) * 1e-3) / 1e9, 1),
+        "dc_frac_measured_min": round(min(v["dc_frac_measured"] for v in sweep.values()), 4),
+        "dc_frac_8tbs_min": round(min(v["dc_frac_8tbs"] for v in sweep.values()), 4),
+        "spread_vs_maxvio": round(spread, 4) if spread is not None else None,
+        "sweep": sweep,
+        "roofline": roofline,
+        "gpu_launches": 4 * args.steps,
+        "clocks": clk,
+    }
+
+    if not args.no_legs:
+        result["legs"] = run_legs(args, dev, world)
+    if not args.no_e2e:
+        result["e2e"] = run_e2e(args, h, plan, w, routes, dev, stream, world)
+    h.close()
+    return result, routes
+
+
+def run_legs(args, dev, world):
+    """prefetch_weight at the inference shape and reduce_grad at the backward
+    shape, timed with CUDA events (median of reps)."""
+    import torch
+    from load_balancing_planner_b200 import moonep
+    legs = {}
+    peak, _ = peaks()
+    R, S, K, E, H, Hp, tp = 8, 4096, 8, 256, 7168, 2048, 128
+    gen = torch.Generator(device=dev).manual_seed(args.seed)
+    reps = 5
+
+    def timed(fn):
+        ts = []
+        for _ in range(reps + 1):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts[1:])
+
+    # prefetch_weight: inference, B = 4, three projections
+    h = moonep.moonep_create(S, H, K, E, R, 4, tp, mode=1)
+    Ws = [torch.randn((E, H, Hp), generator=gen, device=dev, dtype=torch.bfloat16) for _ in range(3)]
+    pools = [torch.empty((R, 4, H, Hp), dtype=torch.bfloat16, device=dev) for _ in range(3)]
+    out = {}
+    for mv in (1.0, 4.0):
+        tk, real, _ = synth.routing(R, S, K, E, mv, "hot8", seed=args.seed)
+        p = moonep.moonep_plan(h, torch.from_numpy(tk).to(dev), torch.from_numpy(synth.local_counts(tk, E)).to(dev))
+        torch.cuda.synchronize()
+        se = p.slots().cpu().numpy()
+        U = int((se >= 0).sum())
+        D = int(np.unique(se[se >= 0]).size)
+        ms = timed(lambda: moonep.moonep_prefetch_weight(h, p, Ws, pools))
+        by = 3 * (D + U) * H * Hp * 2
+        out[f"{mv:g}"] = dict(realised_maxvio=round(real, 4), used_slots=U, distinct_experts=D,
+                              us=round(ms * 1e3, 1), gbs=round(by / (ms * 1e-3) / 1e9, 1),
+                              frac_measured=round(by / (ms * 1e-3) / 1e9 / peak, 4))
+    legs["prefetch_weight"] = dict(workload="inference R=8 S=4096 K=8 E=256 B=4 H=7168 H'=2048, 3 projections",
+                                   bytes="3*(D+U)*H*H'*2", points=out)
+    del Ws, pools
+    h.close()
+
+    # reduce_grad: training plan at maxvio 2, one fp32 projection
+    h = moonep.moonep_create(S, H, K, E, R, 32, tp, mode=0)
+    tk, real, _ = synth.routing(R, S, K, E, 2.0, "hot8", seed=args.seed)
+    p = moonep.moonep_plan(h, torch.from_numpy(tk).to(dev), torch.from_numpy(synth.local_counts(tk, E)).to(dev))
+    G = torch.randn((E, H, Hp), generator=gen, device=dev).mul_(1e-3)
+    RB = torch.randn((R, 32, H, Hp), generator=gen, device=dev).mul_(1e-3)
+    torch.cuda.synchronize()
+    se = p.slots().cpu().numpy()
+    U = int((se >= 0).sum())
+    D = int(np.unique(se[se >= 0]).size)
+    ms = timed(lambda: moonep.moonep_reduce_grad(h, p, [G], [RB]))
+    by = (2 * D + 2 * U) * H * Hp * 4
+    legs["reduce_grad"] = dict(workload="backward E=256 R=8 B=32 H=7168 H'=2048 fp32, plan at maxvio 2",
+                               bytes="(2D+2U)*H*H'*4", realised_maxvio=round(real, 4), used_slots=U,
+                               distinct_experts=D, us=round(ms * 1e3, 1),
+                               gbs=round(by / (ms * 1e-3) / 1e9, 1),
+                               frac_measured=round(by / (ms * 1e-3) / 1e9 / peak, 4))
+    del G, RB
+    h.close()
+    torch.cuda.empty_cache()
+    return legs
+
+
+def run_e2e(args, h, plan, w, routes, dev, stream, world):
+    """The same step through the C ABI from pinned host buffers: H2D of the
+    step's inputs, plan, dispatch, combine, D2H of the combined output."""
+    import torch
+    from load_balancing_planner_b200 import moonep
+    R, S, K, E, H = w["R"], w["S"], w["K"], w["E"], w["H"]
+    nvs = h.nvs
+    hid_h = synth.hidden_bf16(R, S, H, args.seed).pin_memory()
+    wts_h = torch.from_numpy(synth.route_weights(R, S, K, args.seed)).pin_memory()
+    tks_h = [r["topk"].cpu().pin_memory() for r in routes]
+    tpe_h = [r["tpe"].cpu().pin_memory() for r in routes]
+    out_h = torch.empty((R, S, H), dtype=torch.bfloat16).pin_memory()
+    hid_d = torch.empty((R, S, H), dtype=torch.bfloat16, device=dev)
+    wts_d = torch.empty((R, S, K), dtype=torch.float32, device=dev)
+    tk_d = torch.empty((R, S, K), dtype=torch.int32, device=dev)
+    tpe_d = torch.empty((R, E), dtype=torch.int32, device=dev)
+    buf = torch.empty((R, nvs, H), dtype=torch.bfloat16, device=dev)
+    wn = torch.empty((R, nvs), dtype=torch.float32, device=dev)
+    out = torch.empty((R, S, H), dtype=torch.bfloat16, device=dev)
+
+    def step(i):
+        j = i % len(routes)
+        hid_d.copy_(hid_h, non_blocking=True)
+        wts_d.copy_(wts_h, non_blocking=True)
+        tk_d.copy_(tks_h[j], non_blocking=True)
+        tpe_d.copy_(tpe_h[j], non_blocking=True)
+        moonep.moonep_plan(h, tk_d, tpe_d, plan)
+        moonep.moonep_dispatch(h, plan, hid_d, wts_d, buf, wn)
+        moonep.moonep_combine(h, plan, buf, wn, out, None, gather=False)
+        out_h.copy_(out, non_blocking=True)
+
+    n = max(5, min(args.steps, 2 * len(routes)))
+    for i in range(2):
+        step(i)
+    barrier(world)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(n):
+        step(i)
+    b.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(a.elapsed_time(b), world)
+    db, cb = dc_bytes(R, S, K, H)
+    h2d = hid_h.numel() * 2 + wts_h.numel() * 4 + tks_h[0].numel() * 4 + tpe_h[0].numel() * 4
+    return {"value": round(world * (db + cb) * n / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(out_h.numel() * 2),
+            "ms_per_step": round(ms / n, 3), "steps": n}
+
+
+# ---------------------------------------------------------------- the oracle
+def oracle_sample(w, routes_np, ranks_sampled, seed):
+    """Time the CPU oracle as it stands on one host core: the full plan of
+    every routing, then dispatch and combine of every token of the first
+    `ranks_sampled` source ranks (their slots remapped to a compact buffer).
+    Returns (dispatch+combine bytes, seconds)."""
+    import torch
+
+    import oracle
+    R, S, K, E, B, H, tp = w["R"], w["S"], w["K"], w["E"], w["B"], w["H"], w["tp"]
+    n = ranks_sampled
+    x = synth.bf16_bits(torch.from_numpy(synth.normal_f32((n, S, H), seed)).to(torch.bfloat16))
+    wts = synth.route_weights(n, S, K, seed)
+    total_b, total_s = 0, 0.0
+    for tk in routes_np:
+        t0 = time.perf_counter()
+        p = oracle.plan(tk, E, B, tp, w["mode"], synth.local_counts(tk, E))
+        d = p["dst"][:n]
+        # compact slot numbering of the sampled picks, in the plan's own slot order
+        order = np.argsort(d.reshape(-1), kind="stable")
+        comp = np.empty(d.size, np.int32)
+        comp[order] = np.arange(d.size, dtype=np.int32)
+        comp = comp.reshape(d.shape)
+        buf, wn = oracle.dispatch(comp, x, wts, d.size // n)
+        oracle.combine(comp, buf, wn)
+        total_s += time.perf_counter() - t0
+        db, cb = dc_bytes(n, S, K, H)
+        total_b += db + cb
+    return total_b, total_s
+
+
+def cpu_baseline(w, routes, seed):
+    ranks = 2
+    b, s = oracle_sample(w, [r["topk_np"] for r in routes], ranks, seed)
+    return {"value": round(b / s / 1e9, 3), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"full plan of each of the {len(routes)} routings (all {w['R']} ranks) + dispatch and "
+                      f"combine of every token of {ranks} of {w['R']} source ranks, single-threaded C, "
+                      f"{s:.1f} s", "host_cores_available": os.cpu_count()}
+
+
+# ---------------------------------------------------------------- reference arm
+def run_reference(args, world, rank):
+    """The base contract's reference arm is the CPU oracle here: each step is a
+    bounded sample of the same workload (full plan + dispatch/combine of one
+    source rank's tokens) timed on the host."""
+    if rank != 0:
+        return None
+    w = WORKLOADS[args.config]
+    routes = []
+    for mv in w["maxvio"]:
+        tk, real, _ = synth.routing(w["R"], w["S"], w["K"], w["E"], mv, w["profile"], seed=args.seed)
+        routes.append(tk)
+    for i in range(args.warmup):
+        oracle_sample(w, [routes[i % len(routes)]], 1, args.seed)
+    tb, ts = 0, 0.0
+    for i in range(args.steps):
+        b, s = oracle_sample(w, [routes[i % len(routes)]], 1, args.seed)
+        tb += b
+        ts += s
+    v = round(tb / ts / 1e9, 3)
+    return {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ts / args.steps * 1e3, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": f"{args.config}: " + describe(w), "maxvio": list(w["maxvio"])},
+        "cpu_baseline": {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": "per step: full plan of one routing (all ranks) + dispatch and combine of "
+                                   "every token of 1 source rank, single-threaded C"},
+        "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--config", choices=tuple(WORKLOADS), default="train")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-legs", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="ncu DRAM bytes per launch of the dominant kernel, if measured for this build")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        res = run_reference(args, world, rank)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+
+    world, rank, local = setup_dist(args)
+    result, routes = run_ours(args, world, rank, local)
+    if rank == 0 and world == 1 and not args.no_cpu:
+        result["cpu_baseline"] = cpu_baseline(WORKLOADS[args.config], routes, args.seed)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -60,6 +60,7 @@ typedef struct CUstream_st *moonep_stream_t;
 #define MOONEP_STATUS_DUP_EXPERT 2     /* an expert picked twice by one token */
 #define MOONEP_STATUS_COUNT_MISMATCH 4 /* tokens_per_expert differs from the picks */
 #define MOONEP_STATUS_BAD_PLAN 8       /* a plan index pointed outside its buffer; skipped */
+#define MOONEP_STATUS_TIMEOUT 16       /* the planner's grid barrier gave up waiting; destroy the handle */
 
 /* Supported ranges (moonep_create checks them). */
 #define MOONEP_MAX_R 64
@@ -207,6 +208,11 @@ MOONEP_API int moonep_read_status(const moonep_plan_t *plan, int32_t *status, mo
 
 /* Static description of a MOONEP_ERR_* code. */
 MOONEP_API const char *moonep_error_string(int code);
+
+/* Name and text of the CUDA error behind the calling thread's last
+ * MOONEP_ERR_CUDA ("no error" if none yet).  Valid until the next failing call
+ * on this thread. */
+MOONEP_API const char *moonep_last_error(void);
 
 #ifdef __cplusplus
 }

@@ -1,12 +1,12 @@
 // C ABI of libmoonep: host-side validation, the handle, and kernel launches.
 // Every entry point is declared and documented in include/moonep.h.
+#include <stdio.h>
 #include <stdlib.h>
 #include <string.h>
 
 #include "moonep_internal.cuh"
 
 namespace moonep {
-cudaError_t plan_set_smem_limit(size_t bytes);
 cudaError_t weights_set_smem_limit(size_t bytes);
 }  // namespace moonep
 
@@ -17,6 +17,7 @@ struct moonep_handle {
     Dims d;
     int device;
     int sms;            // SMs the copy kernels may occupy
+    int grid_plan;      // planner blocks (all resident)
     int grid_dispatch;  // whole waves over those SMs
     int grid_combine;
     int grid_weights;
@@ -26,10 +27,14 @@ struct moonep_handle {
 
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+static thread_local char g_last_error[256] = "no error";
+
 static int fail_cuda(cudaError_t e) {
-    (void)e;
+    snprintf(g_last_error, sizeof(g_last_error), "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
     return MOONEP_ERR_CUDA;
 }
+
+extern "C" const char *moonep_last_error(void) { return g_last_error; }
 
 extern "C" const char *moonep_error_string(int code) {
     switch (code) {
@@ -82,7 +87,6 @@ extern "C" int moonep_create(const moonep_config_t *cfg, moonep_handle_t *out) {
     d.S = cfg->S; d.H = cfg->H; d.K = cfg->K; d.E = cfg->E; d.R = cfg->R; d.B = cfg->B;
     d.tp = cfg->token_padding; d.mode = cfg->mode;
     d.G = d.E / d.R;
-    d.nch = (d.S + kChunkTokens - 1) / kChunkTokens;
     d.NR = d.E + d.B;
     d.nvs = (int)nvs_of(*cfg);
 
@@ -92,13 +96,43 @@ extern "C" int moonep_create(const moonep_config_t *cfg, moonep_handle_t *out) {
     if (e != cudaSuccess) { free(h); return fail_cuda(e); }
     h->sms = (cfg->num_sms > 0 && cfg->num_sms < sms) ? cfg->num_sms : sms;
 
-    const size_t smem = plan_count_smem_bytes(d);
-    if (smem > 227 * 1024) { free(h); return MOONEP_ERR_CONFIG; }
-    if (smem > 48 * 1024 && (e = plan_set_smem_limit(smem)) != cudaSuccess) { free(h); return fail_cuda(e); }
+    // Planner chunking: every block of the cooperative launch must be resident,
+    // so grow the chunk until R * ceil(S / ct) blocks fit on the device.
+    int smem_optin = 0;
+    if ((e = cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, h->device)) != cudaSuccess) {
+        free(h);
+        return fail_cuda(e);
+    }
+    const size_t smem_max = (size_t)smem_optin - plan_static_smem_bytes();
+    d.ct = d.S < kChunkTokensMin ? d.S : kChunkTokensMin;
+    bool fits = false;
+    for (int iter = 0; iter < 8 && !fits; ++iter) {
+        d.nch = (d.S + d.ct - 1) / d.ct;
+        // as many counting warps as shared memory allows (their per-expert
+        // counters and lane masks grow with E)
+        d.cw = kPlanWarps;
+        while (d.cw > 1 && plan_smem_bytes(d) > smem_max) d.cw /= 2;
+        const size_t smem = plan_smem_bytes(d);
+        if (smem > smem_max || (int64_t)d.ct * d.K > 65535) break;
+        if ((e = plan_set_smem_limit(smem)) != cudaSuccess) { free(h); return fail_cuda(e); }
+        const int cap = plan_blocks_per_sm(d) * sms;
+        if (d.R * d.nch <= cap) {
+            fits = true;
+            break;
+        }
+        if (cap < d.R) break;
+        const int per_rank = cap / d.R;
+        int ct = (d.S + per_rank - 1) / per_rank;
+        ct = (ct + 31) / 32 * 32;
+        d.ct = ct > d.ct ? ct : d.ct + 32;
+    }
+    if (!fits) { free(h); return MOONEP_ERR_CONFIG; }
+    h->grid_plan = d.R * d.nch;
+
     const size_t wsmem = sizeof(int32_t) * 3 * (size_t)d.R * d.B;
     if (wsmem > 48 * 1024 && (e = weights_set_smem_limit(wsmem)) != cudaSuccess) { free(h); return fail_cuda(e); }
 
-    h->grid_dispatch = h->sms * dispatch_blocks_per_sm();
+    h->grid_dispatch = h->sms * dispatch_blocks_per_sm(d.K);
     h->grid_combine = h->sms * combine_blocks_per_sm(d.K);
     h->grid_weights = h->sms * weights_blocks_per_sm();
 
@@ -140,7 +174,7 @@ extern "C" int moonep_plan(moonep_handle_t h, const int32_t *topk, const int32_t
     a.tpe = tokens_per_expert;
     a.plan = *plan;
     a.ws = h->ws;
-    const cudaError_t e = launch_plan(a, h->sms, reinterpret_cast<cudaStream_t>(stream));
+    const cudaError_t e = launch_plan(a, h->grid_plan, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? MOONEP_OK : fail_cuda(e);
 }
 

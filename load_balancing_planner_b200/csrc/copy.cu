@@ -16,11 +16,14 @@ __device__ __forceinline__ uint4 ld_stream(const uint4 *p) { return __ldcs(p); }
 __device__ __forceinline__ void st_stream(uint4 *p, const uint4 &v) { __stcs(p, v); }
 
 // ---- dispatch ----------------------------------------------------------------
-template <int U>
+// KT > 0: K known at compile time, the K destination rows are broadcast into
+// registers once per token; KT == 0: any K, one shuffle per row and step.
+template <int KT, int U>
 __global__ void __launch_bounds__(256) dispatch_kernel(CopyArgs a) {
     pdl_wait();
     if (*a.status != 0) return;
     const Dims &d = a.d;
+    const int K = KT > 0 ? KT : d.K;
     const int lane = threadIdx.x & 31;
     const int HV = d.H >> 3;
     const int64_t ntok = (int64_t)d.R * d.S;
@@ -30,31 +33,57 @@ __global__ void __launch_bounds__(256) dispatch_kernel(CopyArgs a) {
     const int64_t wstride = ((int64_t)gridDim.x * blockDim.x) >> 5;
     for (int64_t tok = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; tok < ntok; tok += wstride) {
         int dk = -1;
-        if (lane < d.K) {
-            dk = a.dst[tok * d.K + lane];
+        if (lane < K) {
+            dk = a.dst[tok * K + lane];
             if (dk < 0 || dk >= nslots) {
                 atomicOr(a.status_rw, MOONEP_STATUS_BAD_PLAN);
                 dk = -1;
             } else if (a.w != nullptr && a.w_out != nullptr) {
-                a.w_out[dk] = __ldcs(a.w + tok * d.K + lane);
+                a.w_out[dk] = __ldcs(a.w + tok * K + lane);
             }
         }
         const uint4 *row = src + tok * HV;
-        for (int v0 = 0; v0 < HV; v0 += 32 * U) {
-            uint4 x[U];
+        if constexpr (KT > 0) {
+            uint4 *orow[KT];
 #pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int v = v0 + u * 32 + lane;
-                if (v < HV) x[u] = ld_stream(row + v);
-            }
-            for (int k = 0; k < d.K; ++k) {
+            for (int k = 0; k < KT; ++k) {
                 const int dd = __shfl_sync(0xffffffffu, dk, k);
-                if (dd < 0) continue;
-                uint4 *o = buf + (int64_t)dd * HV;
+                orow[k] = dd < 0 ? nullptr : buf + (int64_t)dd * HV;
+            }
+            for (int v0 = 0; v0 < HV; v0 += 32 * U) {
+                uint4 x[U];
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
                     const int v = v0 + u * 32 + lane;
-                    if (v < HV) st_stream(o + v, x[u]);
+                    if (v < HV) x[u] = ld_stream(row + v);
+                }
+#pragma unroll
+                for (int k = 0; k < KT; ++k) {
+                    if (orow[k] == nullptr) continue;
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        const int v = v0 + u * 32 + lane;
+                        if (v < HV) st_stream(orow[k] + v, x[u]);
+                    }
+                }
+            }
+        } else {
+            for (int v0 = 0; v0 < HV; v0 += 32 * U) {
+                uint4 x[U];
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int v = v0 + u * 32 + lane;
+                    if (v < HV) x[u] = ld_stream(row + v);
+                }
+                for (int k = 0; k < K; ++k) {
+                    const int dd = __shfl_sync(0xffffffffu, dk, k);
+                    if (dd < 0) continue;
+                    uint4 *o = buf + (int64_t)dd * HV;
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        const int v = v0 + u * 32 + lane;
+                        if (v < HV) st_stream(o + v, x[u]);
+                    }
                 }
             }
         }
@@ -187,15 +216,30 @@ static cudaError_t launch_pdl(Kern kern, int grid, cudaStream_t st, const CopyAr
     return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
-constexpr int kDispatchU = 4;
+#ifndef MOONEP_DISPATCH_U
+#define MOONEP_DISPATCH_U 4
+#endif
+constexpr int kDispatchU = MOONEP_DISPATCH_U;
+
+#define MOONEP_DISPATCH_CASES(X) X(1) X(2) X(4) X(6) X(8)
 
 cudaError_t launch_dispatch(const CopyArgs &a, int grid, cudaStream_t st) {
-    return launch_pdl(dispatch_kernel<kDispatchU>, grid, st, a);
+    switch (a.d.K) {
+#define X(k) case k: return launch_pdl(dispatch_kernel<k, kDispatchU>, grid, st, a);
+        MOONEP_DISPATCH_CASES(X)
+#undef X
+        default: return launch_pdl(dispatch_kernel<0, kDispatchU>, grid, st, a);
+    }
 }
 
-int dispatch_blocks_per_sm() {
+int dispatch_blocks_per_sm(int K) {
     int n = 0;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, dispatch_kernel<kDispatchU>, 256, 0);
+    switch (K) {
+#define X(k) case k: cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, dispatch_kernel<k, kDispatchU>, 256, 0); break;
+        MOONEP_DISPATCH_CASES(X)
+#undef X
+        default: cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, dispatch_kernel<0, kDispatchU>, 256, 0); break;
+    }
     return n > 0 ? n : 1;
 }
 

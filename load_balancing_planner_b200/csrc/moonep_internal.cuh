@@ -5,36 +5,33 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/moonep.h"
+#include "moonep.h"
 
 namespace moonep {
 
-// Planner launch shape: one histogram block per chunk of kChunkTokens tokens
-// of one source rank; the last block to finish also lays the plan out.
-constexpr int kChunkTokens = 512;
-constexpr int kPlanThreads = 512;
+// Planner launch shape: one cooperative block per chunk of `ct` tokens of one
+// source rank (all blocks resident), kPlanThreads threads each.
+constexpr int kPlanThreads = 1024;
 constexpr int kPlanWarps = kPlanThreads / 32;
-constexpr int kDstThreads = 256;
+constexpr int kChunkTokensMin = 512;
+constexpr uint32_t kBarrierPolls = 1u << 22;  // each poll is an L2 round trip: ~2 s, then MOONEP_STATUS_TIMEOUT
 
 struct Dims {
     int S, H, K, E, R, B, tp, mode;
     int G;    // E / R
-    int nch;  // chunks per rank = ceil(S / kChunkTokens)
+    int ct;   // tokens per planner chunk
+    int cw;   // planner warps that count picks (each keeps per-expert counters)
+    int nch;  // chunks per rank = ceil(S / ct)
     int NR;   // rows per rank = E + B
     int nvs;  // NvS
 };
 
-// Planning workspace, carved out of one device allocation owned by the handle.
+// Planning workspace (one device allocation owned by the handle).
 struct Workspace {
-    int32_t *hist;      // [R*nch][E]: chunk histograms, then their exclusive prefix over (r, chunk)
-    uint32_t *arrive;   // [1] blocks of the counting kernel that finished (reset by the last)
-    int32_t *status;    // [1] error bits gathered while counting (reset by the last block)
-    int32_t *estart;    // [E] start of each expert inside its group's sequence
-    int32_t *keep;      // [R] picks each home group keeps
-    int32_t *don;       // [4][R]: donor, recipient, start, length of each donation
-    int32_t *ndon;      // [1]
-    int32_t *rowmap;    // [R][G]: row, on rank s, of the j-th expert of the group s takes from
-    int32_t *rowstart;  // [R][E+B]: first slot of each row
+    int32_t *hist;                // [R*nch][E] picks per (chunk, expert)
+    int32_t *cnt;                 // [2][R][E] picks per (source rank, expert), by call parity
+    unsigned long long *arrive;   // planner blocks that ever reached the grid barrier
+    int32_t *status;              // [2] error bits of the counting phase, by call parity
 };
 
 size_t workspace_bytes(const Dims &d);
@@ -48,8 +45,11 @@ struct PlanArgs {
     Workspace ws;
 };
 
-size_t plan_count_smem_bytes(const Dims &d);
-cudaError_t launch_plan(const PlanArgs &a, int sms, cudaStream_t st);
+size_t plan_smem_bytes(const Dims &d);
+int plan_blocks_per_sm(const Dims &d);
+cudaError_t plan_set_smem_limit(size_t bytes);
+size_t plan_static_smem_bytes();
+cudaError_t launch_plan(const PlanArgs &a, int grid, cudaStream_t st);
 
 struct CopyArgs {
     Dims d;
@@ -64,7 +64,7 @@ struct CopyArgs {
 
 cudaError_t launch_dispatch(const CopyArgs &a, int grid, cudaStream_t st);
 cudaError_t launch_combine(const CopyArgs &a, int grid, cudaStream_t st);
-int dispatch_blocks_per_sm();
+int dispatch_blocks_per_sm(int K);
 int combine_blocks_per_sm(int K);
 
 struct WeightArgs {

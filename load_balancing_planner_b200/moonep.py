@@ -23,7 +23,10 @@ TRAINING, INFERENCE = 0, 1
 
 class MoonepError(RuntimeError):
     def __init__(self, code: int, what: str):
-        super().__init__(f"{what}: {error_string(code)} ({code})")
+        msg = f"{what}: {error_string(code)} ({code})"
+        if code == ERR_CUDA:
+            msg += f" [{lib.moonep_last_error().decode()}]"
+        super().__init__(msg)
         self.code = code
 
 
@@ -54,6 +57,7 @@ def _load():
         "moonep_reduce_grad": ([P, ctypes.POINTER(PlanStruct), i32, P, P, i64, P], ctypes.c_int),
         "moonep_read_status": ([ctypes.POINTER(PlanStruct), ctypes.POINTER(i32), P], ctypes.c_int),
         "moonep_error_string": ([ctypes.c_int], ctypes.c_char_p),
+        "moonep_last_error": ([], ctypes.c_char_p),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -65,7 +69,7 @@ def _load():
 lib = _load()
 EXPORTS = ("moonep_create", "moonep_destroy", "moonep_nvs", "moonep_get_config", "moonep_plan",
            "moonep_dispatch", "moonep_combine", "moonep_prefetch_weight", "moonep_reduce_grad",
-           "moonep_read_status", "moonep_error_string")
+           "moonep_read_status", "moonep_error_string", "moonep_last_error")
 
 
 def error_string(code: int) -> str:

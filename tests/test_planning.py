@@ -95,3 +95,29 @@ def test_golden_plans_on_gpu(cuda):
             else:
                 assert np.array_equal(np.asarray(got[key]), np.asarray(want)), (f, key, np.asarray(got[key]).tolist())
         h.close()
+
+
+def test_random_small_plans_match_oracle(cuda):
+    # 300 random small problems (ranks, group sizes, K, padding, modes, skews):
+    # every donation pattern the alias chain can produce on few ranks
+    from load_balancing_planner_b200 import moonep
+    g = np.random.default_rng(2024)
+    for it in range(300):
+        R = int(g.integers(1, 9))
+        G = int(g.integers(1, 5))
+        E = R * G
+        K = int(g.integers(1, min(E, 4) + 1))
+        S = int(g.integers(1, 41))
+        tp = int(g.integers(1, 5))
+        mode = int(g.integers(0, 2))
+        B = int(g.integers(G, G + 2)) if mode == 0 else int(g.integers(0, G + 1))
+        w = np.ones(E)
+        w[g.integers(0, E)] += g.uniform(0, 4) * E
+        tk = np.stack([g.choice(E, size=K, replace=False, p=w / w.sum()) for _ in range(R * S)])
+        tk = tk.reshape(R, S, K).astype(np.int32)
+        want = oracle.plan(tk, E, B, tp, mode)
+        assert want["status"] == 0
+        h = moonep.moonep_create(S, 8, K, E, R, B, tp, mode=mode)
+        got = plan_to_numpy(gpu_plan(h, tk))
+        assert_plans_equal(got, want)
+        h.close()
