@@ -4,10 +4,13 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "moonep_internal.cuh"
 
 namespace moonep {
 cudaError_t weights_set_smem_limit(size_t bytes);
+size_t weights_static_smem_bytes();
 }  // namespace moonep
 
 using namespace moonep;
@@ -29,10 +32,12 @@ static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 static thread_local char g_last_error[256] = "no error";
 
-static int fail_cuda(cudaError_t e) {
+namespace moonep {
+int fail_cuda(cudaError_t e) {
     snprintf(g_last_error, sizeof(g_last_error), "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
     return MOONEP_ERR_CUDA;
 }
+}  // namespace moonep
 
 extern "C" const char *moonep_last_error(void) { return g_last_error; }
 
@@ -48,13 +53,14 @@ extern "C" const char *moonep_error_string(int code) {
     }
 }
 
-static int64_t nvs_of(const moonep_config_t &c) {
+namespace moonep {
+int64_t nvs_of(const moonep_config_t &c) {
     const int64_t C = (int64_t)c.S * c.K, G = c.E / c.R, tp = c.token_padding;
     const int64_t n = C + 2 * G * (tp - 1);
     return (n + tp - 1) / tp * tp;
 }
 
-static int check_config(const moonep_config_t &c) {
+int check_config(const moonep_config_t &c) {
     if (c.R < 1 || c.R > MOONEP_MAX_R) return MOONEP_ERR_CONFIG;
     if (c.E < 1 || c.E > MOONEP_MAX_E || c.E % c.R != 0) return MOONEP_ERR_CONFIG;
     if (c.K < 1 || c.K > MOONEP_MAX_K || c.K > c.E) return MOONEP_ERR_CONFIG;
@@ -69,9 +75,67 @@ static int check_config(const moonep_config_t &c) {
     return MOONEP_OK;
 }
 
-static bool plan_ok(const moonep_plan_t *p) {
+// Raise the dynamic shared-memory limit of the kernels that need more than
+// 48 KB to the device's maximum, once per device (a per-function attribute:
+// setting it per handle would let a later small handle lower it below an
+// earlier large handle's need).
+int prepare_device(int device) {
+    static std::mutex mu;
+    static bool done[kMaxDevices] = {};
+    if (device < 0 || device >= kMaxDevices) return MOONEP_ERR_SIZE;
+    std::lock_guard<std::mutex> lock(mu);
+    if (done[device]) return MOONEP_OK;
+    int optin = 0;
+    cudaError_t e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
+    if (e == cudaSuccess) e = plan_set_smem_limit((size_t)optin - plan_static_smem_bytes());
+    if (e == cudaSuccess) e = weights_set_smem_limit((size_t)optin - weights_static_smem_bytes());
+    if (e != cudaSuccess) return fail_cuda(e);
+    done[device] = true;
+    return MOONEP_OK;
+}
+
+// Planner dimensions for cfg on `device`: every block of the cooperative
+// launch must be resident, so the chunk grows until R * ceil(S / ct) blocks
+// fit; the counting warps shrink until their per-expert tables fit.
+int plan_dims(const moonep_config_t &cfg, int device, Dims *out, int *grid) {
+    Dims d;
+    memset(&d, 0, sizeof(d));
+    d.S = cfg.S; d.H = cfg.H; d.K = cfg.K; d.E = cfg.E; d.R = cfg.R; d.B = cfg.B;
+    d.tp = cfg.token_padding; d.mode = cfg.mode;
+    d.G = d.E / d.R;
+    d.NR = d.E + d.B;
+    d.nvs = (int)nvs_of(cfg);
+    int sms = 0, optin = 0;
+    cudaError_t e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
+    if (e != cudaSuccess) return fail_cuda(e);
+    const size_t smem_max = (size_t)optin - plan_static_smem_bytes();
+    d.ct = d.S < kChunkTokensMin ? d.S : kChunkTokensMin;
+    for (int iter = 0; iter < 8; ++iter) {
+        d.nch = (d.S + d.ct - 1) / d.ct;
+        d.cw = kPlanWarps;
+        while (d.cw > 1 && plan_smem_bytes(d) > smem_max) d.cw /= 2;
+        if (plan_smem_bytes(d) > smem_max || (int64_t)d.ct * d.K > 65535) return MOONEP_ERR_CONFIG;
+        const int cap = plan_blocks_per_sm(d) * sms;
+        if (d.R * d.nch <= cap) {
+            *out = d;
+            *grid = d.R * d.nch;
+            return MOONEP_OK;
+        }
+        if (cap < d.R) return MOONEP_ERR_CONFIG;
+        const int per_rank = cap / d.R;
+        int ct = (d.S + per_rank - 1) / per_rank;
+        ct = (ct + 31) / 32 * 32;
+        d.ct = ct > d.ct ? ct : d.ct + 32;
+    }
+    return MOONEP_ERR_CONFIG;
+}
+
+bool plan_ok(const moonep_plan_t *p) {
     return p && p->dst && p->cu_seqlens && p->row_counts && p->counts && p->assign && p->maxvio && p->status;
 }
+}  // namespace moonep
+
 
 extern "C" int moonep_create(const moonep_config_t *cfg, moonep_handle_t *out) {
     if (!out) return MOONEP_ERR_NULL;
@@ -84,53 +148,14 @@ extern "C" int moonep_create(const moonep_config_t *cfg, moonep_handle_t *out) {
     if (!h) return MOONEP_ERR_CUDA;
     h->cfg = *cfg;
     Dims &d = h->d;
-    d.S = cfg->S; d.H = cfg->H; d.K = cfg->K; d.E = cfg->E; d.R = cfg->R; d.B = cfg->B;
-    d.tp = cfg->token_padding; d.mode = cfg->mode;
-    d.G = d.E / d.R;
-    d.NR = d.E + d.B;
-    d.nvs = (int)nvs_of(*cfg);
-
     cudaError_t e = cudaGetDevice(&h->device);
     int sms = 0;
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, h->device);
     if (e != cudaSuccess) { free(h); return fail_cuda(e); }
     h->sms = (cfg->num_sms > 0 && cfg->num_sms < sms) ? cfg->num_sms : sms;
-
-    // Planner chunking: every block of the cooperative launch must be resident,
-    // so grow the chunk until R * ceil(S / ct) blocks fit on the device.
-    int smem_optin = 0;
-    if ((e = cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, h->device)) != cudaSuccess) {
-        free(h);
-        return fail_cuda(e);
-    }
-    const size_t smem_max = (size_t)smem_optin - plan_static_smem_bytes();
-    d.ct = d.S < kChunkTokensMin ? d.S : kChunkTokensMin;
-    bool fits = false;
-    for (int iter = 0; iter < 8 && !fits; ++iter) {
-        d.nch = (d.S + d.ct - 1) / d.ct;
-        // as many counting warps as shared memory allows (their per-expert
-        // counters and lane masks grow with E)
-        d.cw = kPlanWarps;
-        while (d.cw > 1 && plan_smem_bytes(d) > smem_max) d.cw /= 2;
-        const size_t smem = plan_smem_bytes(d);
-        if (smem > smem_max || (int64_t)d.ct * d.K > 65535) break;
-        if ((e = plan_set_smem_limit(smem)) != cudaSuccess) { free(h); return fail_cuda(e); }
-        const int cap = plan_blocks_per_sm(d) * sms;
-        if (d.R * d.nch <= cap) {
-            fits = true;
-            break;
-        }
-        if (cap < d.R) break;
-        const int per_rank = cap / d.R;
-        int ct = (d.S + per_rank - 1) / per_rank;
-        ct = (ct + 31) / 32 * 32;
-        d.ct = ct > d.ct ? ct : d.ct + 32;
-    }
-    if (!fits) { free(h); return MOONEP_ERR_CONFIG; }
-    h->grid_plan = d.R * d.nch;
-
-    const size_t wsmem = sizeof(int32_t) * 3 * (size_t)d.R * d.B;
-    if (wsmem > 48 * 1024 && (e = weights_set_smem_limit(wsmem)) != cudaSuccess) { free(h); return fail_cuda(e); }
+    int rc2 = prepare_device(h->device);
+    if (rc2 == MOONEP_OK) rc2 = plan_dims(*cfg, h->device, &d, &h->grid_plan);
+    if (rc2 != MOONEP_OK) { free(h); return rc2; }
 
     h->grid_dispatch = h->sms * dispatch_blocks_per_sm(d.K);
     h->grid_combine = h->sms * combine_blocks_per_sm(d.K);

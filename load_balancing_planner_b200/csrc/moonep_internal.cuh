@@ -14,6 +14,7 @@ namespace moonep {
 constexpr int kPlanThreads = 1024;
 constexpr int kPlanWarps = kPlanThreads / 32;
 constexpr int kChunkTokensMin = 512;
+constexpr int kMaxDevices = 64;
 constexpr uint32_t kBarrierPolls = 1u << 22;  // each poll is an L2 round trip: ~2 s, then MOONEP_STATUS_TIMEOUT
 
 struct Dims {
@@ -80,6 +81,14 @@ struct WeightArgs {
 cudaError_t launch_prefetch(const WeightArgs &a, int grid, cudaStream_t st);
 cudaError_t launch_reduce_grad(const WeightArgs &a, int grid, cudaStream_t st);
 int weights_blocks_per_sm();
+
+// ---- host helpers shared by the entry points (api.cu) ----------------------
+int fail_cuda(cudaError_t e);                  // records the error text, returns MOONEP_ERR_CUDA
+int64_t nvs_of(const moonep_config_t &c);
+int check_config(const moonep_config_t &c);
+int prepare_device(int device);                // kernel attributes, once per device
+int plan_dims(const moonep_config_t &c, int device, Dims *d, int *grid);
+bool plan_ok(const moonep_plan_t *p);
 
 // ---- small device helpers ------------------------------------------------
 __device__ __forceinline__ unsigned lanemask_lt() {

@@ -234,6 +234,14 @@ int weights_blocks_per_sm() {
     return n > 0 ? n : 1;
 }
 
+size_t weights_static_smem_bytes() {
+    cudaFuncAttributes fa;
+    size_t m = 0;
+    if (cudaFuncGetAttributes(&fa, prefetch_kernel) == cudaSuccess) m = fa.sharedSizeBytes;
+    if (cudaFuncGetAttributes(&fa, reduce_grad_kernel) == cudaSuccess && fa.sharedSizeBytes > m) m = fa.sharedSizeBytes;
+    return m;
+}
+
 cudaError_t weights_set_smem_limit(size_t bytes) {
     cudaError_t e = cudaFuncSetAttribute(prefetch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e != cudaSuccess) return e;
