@@ -156,13 +156,25 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """Largest value over the ranks (a timing, never data of the path)."""
     import torch
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(seed, rank):
+    """Every rank draws its own EP group's inputs: independent problems."""
+    return seed + rank
+
+
+def aggregate_gbs(bytes_per_rank_step, steps, world, max_ms):
+    """Whole-job throughput: the bytes all ranks moved over the slowest rank's time."""
+    return world * bytes_per_rank_step * steps / (max_ms * 1e-3) / 1e9
 
 
 def make_inputs(w, seed, dev):
@@ -188,7 +200,7 @@ def run_ours(args, world, rank, local):
     w = WORKLOADS[args.config]
     R, S, K, E, B, H, tp = w["R"], w["S"], w["K"], w["E"], w["B"], w["H"], w["tp"]
     dev = torch.device("cuda", local if world > 1 else 0)
-    seed = args.seed + rank
+    seed = rank_seed(args.seed, rank)
     hidden, weights, routes = make_inputs(w, seed, dev)
     h = moonep.moonep_create(S, H, K, E, R, B, tp, mode=w["mode"])
     nvs = h.nvs
@@ -242,7 +254,7 @@ def run_ours(args, world, rank, local):
     comb_ms = [e[2].elapsed_time(e[3]) for e in evs]
     db, cb = dc_bytes(R, S, K, H)
     peak, peak_kind = peaks()
-    value = world * (db + cb) * args.steps / (total_ms_max * 1e-3) / 1e9
+    value = aggregate_gbs(db + cb, args.steps, world, total_ms_max)
 
     sweep = {}
     for j, r in enumerate(routes):
@@ -412,7 +424,7 @@ def run_e2e(args, h, plan, w, routes, dev, stream, world):
     ms = max_over_ranks(a.elapsed_time(b), world)
     db, cb = dc_bytes(R, S, K, H)
     h2d = hid_h.numel() * 2 + wts_h.numel() * 4 + tks_h[0].numel() * 4 + tpe_h[0].numel() * 4
-    return {"value": round(world * (db + cb) * n / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+    return {"value": round(aggregate_gbs(db + cb, n, world, ms), 1), "unit": "GB/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(out_h.numel() * 2),
             "ms_per_step": round(ms / n, 3), "steps": n}
 
@@ -449,7 +461,7 @@ def oracle_sample(w, routes_np, ranks_sampled, seed):
 
 
 def cpu_baseline(w, routes, seed):
-    ranks = 2
+    ranks = 4
     b, s = oracle_sample(w, [r["topk_np"] for r in routes], ranks, seed)
     return {"value": round(b / s / 1e9, 3), "unit": "GB/s", "cores": 1, "kind": "oracle",
             "sample": f"full plan of each of the {len(routes)} routings (all {w['R']} ranks) + dispatch and "

@@ -1,0 +1,64 @@
+"""The N-GPU path of bench.py on CPU with gloo, world size 2: every rank runs
+its own independent EP group (different seeds, no data-path collective), the
+timing is the max over ranks, and the value aggregates all ranks' bytes."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import oracle
+from load_balancing_planner_b200 import synth
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, world, port, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    import bench
+    try:
+        # each rank plans its own routing with the oracle (host stand-in for
+        # the device planner): independent problems, nothing exchanged
+        seed = bench.rank_seed(0, rank)
+        tk, mv, _ = synth.routing(4, 64, 4, 16, 1.5, "hot8", seed=seed)
+        p = oracle.plan(tk, 16, 4, 8)
+        t_ms = 10.0 * (rank + 1)
+        tmax = bench.max_over_ranks(t_ms, world)
+        q.put((rank, int(p["status"]), int(p["dst"].sum()), tmax))
+    finally:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def test_two_rank_bench_logic_gloo():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for pr in procs:
+        pr.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for pr in procs:
+        pr.join(timeout=60)
+        assert pr.exitcode == 0
+    (r0, st0, s0, m0), (r1, st1, s1, m1) = res
+    assert st0 == st1 == 0
+    assert s0 != s1, "ranks must draw different problems"
+    assert m0 == m1 == 20.0, "timing is the max over ranks"
+
+
+def test_aggregate_value_counts_all_ranks():
+    import bench
+    assert bench.aggregate_gbs(1e9, 10, 4, 1000.0) == pytest.approx(40.0)
+    assert bench.rank_seed(3, 2) == 5
