@@ -203,6 +203,34 @@ MOONEP_API int moonep_reduce_grad(moonep_handle_t h, const moonep_plan_t *plan, 
                        float *const *grads, float *const *reduce_buffers, int64_t Hp,
                        moonep_stream_t stream);
 
+/*
+ * moonep_plan without a handle and without allocating: the same plan as
+ * moonep_plan for the same cfg and inputs.  (This entry point has no
+ * counterpart on the pages; it exists for callers that cannot call cudaMalloc
+ * in the layer path, e.g. when a caching allocator or a start-up reservation
+ * owns all device memory, where a raw cudaMalloc would break that budget and
+ * may synchronise the device.)
+ *
+ * Its planning workspace is one fixed array of MOONEP_NOALLOC_SCRATCH_BYTES in
+ * device memory, part of the library image: every GPU that loads the library
+ * holds it until the process exits.  A cfg whose workspace does not fit is
+ * rejected with MOONEP_ERR_SIZE (the training shape R=8, S=4096, K=8, E=256
+ * needs about 80 KB).  The call allocates nothing (no cudaMalloc, cudaFree or
+ * allocating library routine); it clears the part of the array that must
+ * start at zero with cudaMemsetAsync on `stream`.
+ *
+ * The first call on a device looks the array's device address up
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture.  All calls share the one array: calls that
+ * overlap on the GPU race, so order them on one stream.  Arguments, layouts
+ * and status bits are those of moonep_plan; cfg is checked as moonep_create
+ * checks it.
+ */
+#define MOONEP_NOALLOC_SCRATCH_BYTES (1 << 20)
+MOONEP_API int moonep_plan_noalloc(const moonep_config_t *cfg, const int32_t *topk,
+                                   const int32_t *tokens_per_expert, const moonep_plan_t *plan,
+                                   moonep_stream_t stream);
+
 /* Read plan->status into *status (host).  Synchronises `stream`. */
 MOONEP_API int moonep_read_status(const moonep_plan_t *plan, int32_t *status, moonep_stream_t stream);
 

@@ -58,6 +58,7 @@ def _load():
         "moonep_read_status": ([ctypes.POINTER(PlanStruct), ctypes.POINTER(i32), P], ctypes.c_int),
         "moonep_error_string": ([ctypes.c_int], ctypes.c_char_p),
         "moonep_last_error": ([], ctypes.c_char_p),
+        "moonep_plan_noalloc": ([ctypes.POINTER(Config), P, P, ctypes.POINTER(PlanStruct), P], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -69,7 +70,8 @@ def _load():
 lib = _load()
 EXPORTS = ("moonep_create", "moonep_destroy", "moonep_nvs", "moonep_get_config", "moonep_plan",
            "moonep_dispatch", "moonep_combine", "moonep_prefetch_weight", "moonep_reduce_grad",
-           "moonep_read_status", "moonep_error_string", "moonep_last_error")
+           "moonep_read_status", "moonep_error_string", "moonep_last_error", "moonep_plan_noalloc")
+NOALLOC_SCRATCH_BYTES = 1 << 20
 
 
 def error_string(code: int) -> str:
@@ -129,9 +131,10 @@ class Handle:
 
 
 class Plan:
-    """Device arrays of one plan (caller-owned, see moonep_plan_t)."""
+    """Device arrays of one plan (caller-owned, see moonep_plan_t).  `h` is a
+    Handle, or a Config for moonep_plan_noalloc."""
 
-    def __init__(self, h: Handle, device=None):
+    def __init__(self, h, device=None):
         dev = device or torch.device("cuda", torch.cuda.current_device())
         R, S, K, E, B = h.R, h.S, h.K, h.E, h.B
         i32 = dict(dtype=torch.int32, device=dev)
@@ -146,7 +149,7 @@ class Plan:
         self.struct = PlanStruct(*(t.data_ptr() for t in (
             self.dst, self.cu_seqlens, self.row_counts, self.slot_expert, self.counts,
             self.assign, self.maxvio, self.status)))
-        self.nvs = h.nvs
+        self.nvs = h.nvs if isinstance(h, Handle) else None
         self.B = B
 
     def slots(self):
@@ -175,6 +178,17 @@ def moonep_plan(h: Handle, topk, tokens_per_expert=None, plan: Plan | None = Non
     plan = plan or Plan(h, topk.device)
     _check(lib.moonep_plan(h.ptr, _ptr(topk), _ptr(tokens_per_expert), ctypes.byref(plan.struct),
                            _stream(stream)), "moonep_plan")
+    return plan
+
+
+def moonep_plan_noalloc(cfg: Config, topk, tokens_per_expert=None, plan: Plan | None = None,
+                        stream=None) -> Plan:
+    """The planner without a handle or any device allocation (see moonep.h)."""
+    _expect(topk, (cfg.R, cfg.S, cfg.K), torch.int32, "topk")
+    _expect(tokens_per_expert, (cfg.R, cfg.E), torch.int32, "tokens_per_expert")
+    plan = plan or Plan(cfg, topk.device)
+    _check(lib.moonep_plan_noalloc(ctypes.byref(cfg), _ptr(topk), _ptr(tokens_per_expert),
+                                   ctypes.byref(plan.struct), _stream(stream)), "moonep_plan_noalloc")
     return plan
 
 
