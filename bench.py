@@ -71,6 +71,25 @@ def dc_bytes(R, S, K, H):
     return disp, comb
 
 
+def recorded_traffic(kernel):
+    """DRAM bytes per launch of `kernel` at the training shape, from the ncu
+    record in profiles/dram_traffic_train.md -- only if that record was taken
+    on the current source of the copy kernels (hash match), else None."""
+    import hashlib
+    import re
+    try:
+        with open(os.path.join(ROOT, "load_balancing_planner_b200", "csrc", "copy.cu"), "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()[:16]
+        with open(os.path.join(ROOT, "profiles", "dram_traffic_train.md")) as f:
+            for line in f:
+                m = re.search(r"traffic: kernel=(\w+) bytes_per_launch=(\d+) copy_cu_sha256=(\w+)", line)
+                if m and m.group(1) == kernel and m.group(3) == sha:
+                    return int(m.group(2))
+    except OSError:
+        pass
+    return None
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -278,7 +297,8 @@ def run_ours(args, world, rank, local):
     roofline = dict(bound="hbm", kernel=dom[0], achieved=round(achieved, 1), peak=peak, unit="GB/s",
                     frac=round(achieved / peak, 4), peak_kind=peak_kind,
                     frac_of_nominal_8tbs=round(achieved / NOMINAL_HBM_GBS, 4),
-                    traffic=args.traffic, bytes_per_launch=dom[2])
+                    traffic=args.traffic if args.traffic is not None else recorded_traffic(dom[0] + "_kernel"),
+                    bytes_per_launch=dom[2])
 
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,

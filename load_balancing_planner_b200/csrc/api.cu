@@ -22,6 +22,7 @@ struct moonep_handle {
     int sms;            // SMs the copy kernels may occupy
     int grid_plan;      // planner blocks (all resident)
     int grid_dispatch;  // whole waves over those SMs
+    bool bulk_dispatch; // rows moved with bulk copies through shared memory
     int grid_combine;
     int grid_weights;
     void *ws_mem;
@@ -89,6 +90,7 @@ int prepare_device(int device) {
     cudaError_t e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
     if (e == cudaSuccess) e = plan_set_smem_limit((size_t)optin - plan_static_smem_bytes());
     if (e == cudaSuccess) e = weights_set_smem_limit((size_t)optin - weights_static_smem_bytes());
+    if (e == cudaSuccess) e = dispatch_bulk_set_smem_limit((size_t)optin - 1024);
     if (e != cudaSuccess) return fail_cuda(e);
     done[device] = true;
     return MOONEP_OK;
@@ -157,7 +159,8 @@ extern "C" int moonep_create(const moonep_config_t *cfg, moonep_handle_t *out) {
     if (rc2 == MOONEP_OK) rc2 = plan_dims(*cfg, h->device, &d, &h->grid_plan);
     if (rc2 != MOONEP_OK) { free(h); return rc2; }
 
-    h->grid_dispatch = h->sms * dispatch_blocks_per_sm(d.K);
+    h->bulk_dispatch = dispatch_use_bulk(d);
+    h->grid_dispatch = h->sms * (h->bulk_dispatch ? dispatch_bulk_blocks_per_sm(d) : dispatch_blocks_per_sm(d.K));
     h->grid_combine = h->sms * combine_blocks_per_sm(d.K);
     h->grid_weights = h->sms * weights_blocks_per_sm();
 
@@ -222,7 +225,9 @@ extern "C" int moonep_dispatch(moonep_handle_t h, const moonep_plan_t *plan, con
     a.w = route_weights;
     a.out = hidden_nvs;
     a.w_out = route_weights_nvs;
-    const cudaError_t e = launch_dispatch(a, h->grid_dispatch, reinterpret_cast<cudaStream_t>(stream));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const cudaError_t e = h->bulk_dispatch ? launch_dispatch_bulk(a, h->grid_dispatch, st)
+                                           : launch_dispatch(a, h->grid_dispatch, st);
     return e == cudaSuccess ? MOONEP_OK : fail_cuda(e);
 }
 

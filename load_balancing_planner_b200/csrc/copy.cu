@@ -90,6 +90,135 @@ __global__ void __launch_bounds__(256) dispatch_kernel(CopyArgs a) {
     }
 }
 
+// ---- dispatch with bulk (TMA) copies -----------------------------------------
+// Rows of at least kBulkMinRow bytes move through shared memory with the bulk
+// copy engine: each warp runs a ring of NS row stages.  Lane 0 loads a token's
+// row with one bulk global->shared copy (completion on an mbarrier), then
+// writes it to its K slots with K bulk shared->global copies (one bulk group
+// per token); a stage is refilled once the previous token's stores have read
+// it.  Waits are bounded: on a timeout the kernel flags MOONEP_STATUS_TIMEOUT,
+// drains what it issued and returns.
+constexpr int kBulkMinRow = 2048;
+constexpr int kBulkStages = 3;
+constexpr uint32_t kBulkPolls = 1u << 22;
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint32_t bar) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+    for (uint32_t it = 0; it < kBulkPolls; ++it) {
+        uint32_t done;
+        asm volatile(
+            "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+            : "=r"(done)
+            : "r"(bar), "r"(parity)
+            : "memory");
+        if (done) return true;
+    }
+    return false;
+}
+// Stores are marked evict-first in L2 (like the streaming stores of the
+// vector path), so the next kernel does not inherit an L2 full of dirty rows.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+__device__ __forceinline__ void bulk_store(void *dst, uint32_t src, uint32_t bytes, uint64_t pol) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group.L2::cache_hint [%0], [%1], %2, %3;" ::"l"(dst), "r"(src),
+                 "r"(bytes), "l"(pol)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// one warp per block; NS stages of `rowbytes` each, then NS mbarriers
+template <int KT>
+__global__ void __launch_bounds__(32) dispatch_bulk_kernel(CopyArgs a) {
+    extern __shared__ __align__(128) uint8_t sm[];
+    pdl_wait();
+    if (*a.status != 0) return;
+    const Dims &d = a.d;
+    const int K = KT > 0 ? KT : d.K;
+    const int lane = threadIdx.x;
+    const uint32_t rowbytes = (uint32_t)d.H * 2u;
+    const int64_t ntok = (int64_t)d.R * d.S;
+    const int64_t nslots = (int64_t)d.R * d.nvs;
+    const uint8_t *src = static_cast<const uint8_t *>(a.src);
+    uint8_t *buf = static_cast<uint8_t *>(a.out);
+    const uint32_t stage0 = smem_addr(sm);
+    const uint32_t bar0 = smem_addr(sm + (size_t)kBulkStages * rowbytes);
+    const int64_t first = blockIdx.x, step = gridDim.x;
+    auto tok_of = [&](int64_t i) { return first + i * step; };
+    const uint64_t pol = l2_evict_first_policy();
+
+    if (lane == 0) {
+        for (int s = 0; s < kBulkStages; ++s) mbar_init(bar0 + 8u * s);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        for (int s = 0; s < kBulkStages; ++s)
+            if (tok_of(s) < ntok)
+                bulk_load(stage0 + s * rowbytes, src + tok_of(s) * rowbytes, rowbytes, bar0 + 8u * s);
+    }
+    __syncwarp();
+    bool ok = true;
+    int64_t i = 0;
+    for (; tok_of(i) < ntok; ++i) {
+        const int64_t tok = tok_of(i);
+        const int s = (int)(i % kBulkStages);
+        const uint32_t parity = (uint32_t)((i / kBulkStages) & 1);
+        int dk = -1;
+        if (lane < K) {
+            dk = a.dst[tok * K + lane];
+            if (dk < 0 || dk >= nslots) {
+                atomicOr(a.status_rw, MOONEP_STATUS_BAD_PLAN);
+                dk = -1;
+            } else if (a.w != nullptr && a.w_out != nullptr) {
+                a.w_out[dk] = __ldcs(a.w + tok * K + lane);
+            }
+        }
+        if (lane == 0) ok = mbar_wait(bar0 + 8u * s, parity);
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
+        for (int k = 0; k < K; ++k) {
+            const int dd = __shfl_sync(0xffffffffu, dk, k);
+            if (lane == 0 && dd >= 0) bulk_store(buf + (int64_t)dd * rowbytes, stage0 + s * rowbytes, rowbytes, pol);
+        }
+        if (lane == 0) {
+            bulk_commit();
+            // refill the previous token's stage once its stores have read it
+            if (i >= 1 && tok_of(i - 1 + kBulkStages) < ntok) {
+                bulk_wait_read1();
+                const int sp = (int)((i - 1) % kBulkStages);
+                bulk_load(stage0 + sp * rowbytes, src + tok_of(i - 1 + kBulkStages) * rowbytes, rowbytes,
+                          bar0 + 8u * sp);
+            }
+        }
+        __syncwarp();
+    }
+    if (lane == 0) {
+        if (!ok) {
+            atomicOr(a.status_rw, MOONEP_STATUS_TIMEOUT);
+            // loads still in flight: tokens i .. i + kBulkStages - 2 (bounded waits)
+            for (int64_t j = i; j < i + kBulkStages - 1 && tok_of(j) < ntok; ++j)
+                mbar_wait(bar0 + 8u * (uint32_t)(j % kBulkStages), (uint32_t)((j / kBulkStages) & 1));
+        }
+        bulk_wait_all();  // every issued load was consumed; the stores must finish reading
+    }
+    __syncwarp();
+}
+
+size_t dispatch_bulk_smem(const Dims &d) { return (size_t)kBulkStages * d.H * 2 + 8 * kBulkStages; }
+bool dispatch_use_bulk(const Dims &d) { return (size_t)d.H * 2 >= kBulkMinRow && dispatch_bulk_smem(d) <= 200 * 1024; }
+
 // ---- combine -----------------------------------------------------------------
 __device__ __forceinline__ void fma_bf16x8(float (&acc)[8], const uint4 &y, float w) {
     const uint32_t q[4] = {y.x, y.y, y.z, y.w};
@@ -223,6 +352,19 @@ constexpr int kDispatchU = MOONEP_DISPATCH_U;
 
 #define MOONEP_DISPATCH_CASES(X) X(1) X(2) X(4) X(6) X(8)
 
+template <typename Kern>
+static cudaError_t launch_pdl_smem(Kern kern, int grid, int block, size_t smem, cudaStream_t st, const CopyArgs &a) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1] = {pdl_attr()};
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
 cudaError_t launch_dispatch(const CopyArgs &a, int grid, cudaStream_t st) {
     switch (a.d.K) {
 #define X(k) case k: return launch_pdl(dispatch_kernel<k, kDispatchU>, grid, st, a);
@@ -230,6 +372,37 @@ cudaError_t launch_dispatch(const CopyArgs &a, int grid, cudaStream_t st) {
 #undef X
         default: return launch_pdl(dispatch_kernel<0, kDispatchU>, grid, st, a);
     }
+}
+
+cudaError_t launch_dispatch_bulk(const CopyArgs &a, int grid, cudaStream_t st) {
+    const size_t smem = dispatch_bulk_smem(a.d);
+    switch (a.d.K) {
+#define X(k) case k: return launch_pdl_smem(dispatch_bulk_kernel<k>, grid, 32, smem, st, a);
+        MOONEP_DISPATCH_CASES(X)
+#undef X
+        default: return launch_pdl_smem(dispatch_bulk_kernel<0>, grid, 32, smem, st, a);
+    }
+}
+
+cudaError_t dispatch_bulk_set_smem_limit(size_t bytes) {
+    cudaError_t e = cudaSuccess;
+#define X(k) if (e == cudaSuccess) e = cudaFuncSetAttribute(dispatch_bulk_kernel<k>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    MOONEP_DISPATCH_CASES(X)
+    X(0)
+#undef X
+    return e;
+}
+
+int dispatch_bulk_blocks_per_sm(const Dims &d) {
+    int n = 0;
+    const size_t smem = dispatch_bulk_smem(d);
+    switch (d.K) {
+#define X(k) case k: cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, dispatch_bulk_kernel<k>, 32, smem); break;
+        MOONEP_DISPATCH_CASES(X)
+#undef X
+        default: cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, dispatch_bulk_kernel<0>, 32, smem); break;
+    }
+    return n > 0 ? n : 1;
 }
 
 int dispatch_blocks_per_sm(int K) {

@@ -64,6 +64,10 @@ struct CopyArgs {
 };
 
 cudaError_t launch_dispatch(const CopyArgs &a, int grid, cudaStream_t st);
+cudaError_t launch_dispatch_bulk(const CopyArgs &a, int grid, cudaStream_t st);
+cudaError_t dispatch_bulk_set_smem_limit(size_t bytes);
+int dispatch_bulk_blocks_per_sm(const Dims &d);
+bool dispatch_use_bulk(const Dims &d);
 cudaError_t launch_combine(const CopyArgs &a, int grid, cudaStream_t st);
 int dispatch_blocks_per_sm(int K);
 int combine_blocks_per_sm(int K);
