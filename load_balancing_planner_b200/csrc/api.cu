@@ -115,6 +115,10 @@ int plan_dims(const moonep_config_t &cfg, int device, Dims *out, int *grid) {
     d.ct = d.S < kChunkTokensMin ? d.S : kChunkTokensMin;
     for (int iter = 0; iter < 8; ++iter) {
         d.nch = (d.S + d.ct - 1) / d.ct;
+        // second-recipient bases only where the layout tables still fit
+        d.cw = 1;
+        d.fast2 = 1;
+        if (plan_smem_bytes(d) > smem_max) d.fast2 = 0;
         d.cw = kPlanWarps;
         while (d.cw > 1 && plan_smem_bytes(d) > smem_max) d.cw /= 2;
         if (plan_smem_bytes(d) > smem_max || (int64_t)d.ct * d.K > 65535) return MOONEP_ERR_CONFIG;

@@ -25,6 +25,7 @@ struct Dims {
     int nch;  // chunks per rank = ceil(S / ct)
     int NR;   // rows per rank = E + B
     int nvs;  // NvS
+    int fast2;  // planner keeps second-recipient dst bases (when shared memory allows)
 };
 
 // Planning workspace (one device allocation owned by the handle).

@@ -53,8 +53,11 @@ __host__ __device__ static inline size_t counts_bytes(const Dims &d) {
 __host__ __device__ static size_t region1_bytes(const Dims &d) {
     // counting phase: per-warp counts + per-warp lane masks; layout phase reuses it
     const size_t counts = counts_bytes(d) + sizeof(uint32_t) * (size_t)d.cw * d.E;
-    const size_t layout = sizeof(int32_t) * (9 * (size_t)d.E + 2 * (size_t)d.R * d.B) +
-                          sizeof(int16_t) * (2 * (size_t)d.E + 2);
+    // int32: T, pre, es, nhome, kbase, nrecv, ovfincl, recvstart, ebase, eend
+    // (10 E), ebase2, eend2 (2 E, when fast2) + slotincl (R B);
+    // int16: qidx (E) + slotj (R B)
+    const size_t layout = sizeof(int32_t) * ((10 + 2 * (size_t)d.fast2) * d.E + (size_t)d.R * d.B) +
+                          sizeof(int16_t) * ((size_t)d.E + (size_t)d.R * d.B + 2);
     return align256(counts > layout ? counts : layout);
 }
 
@@ -62,8 +65,9 @@ __host__ __device__ static size_t region1_bytes(const Dims &d) {
 // checked after the barrier) when they are small enough.
 __host__ __device__ static inline bool tpe_in_smem(const Dims &d) { return (size_t)d.R * d.E <= 16384; }
 
+// picks of the block's chunk: expert (u16) and rank inside the chunk (u16, < ct*K <= 65535)
 __host__ __device__ static inline size_t ent_bytes(const Dims &d) {
-    return align256(sizeof(uint16_t) * (size_t)d.ct * d.K) + align256(sizeof(int32_t) * (size_t)d.ct * d.K);
+    return 2 * align256(sizeof(uint16_t) * (size_t)d.ct * d.K);
 }
 
 size_t plan_smem_bytes(const Dims &d) {
@@ -115,34 +119,170 @@ __device__ __forceinline__ int warp_max(int v) {
 
 __device__ __forceinline__ int pad_to(int n, int tp) { return n ? (n + tp - 1) / tp * tp : 0; }
 
-// Grid barrier over all blocks of a cooperative launch.  The counter only
-// grows: at kernel start it holds k * gridDim.x (k calls done), every block
-// adds one, and all wait until it reaches (k + 1) * gridDim.x, with a bounded
-// number of polls.  Returns false on timeout.
-__device__ bool grid_barrier(unsigned long long *ctr, unsigned long long target) {
+// Grid barrier over all blocks of a cooperative launch, split into arrive and
+// wait so a block can do local work in between.  The counter only grows: at
+// kernel start it holds k * gridDim.x (k calls done), every block adds one,
+// and all wait until it reaches (k + 1) * gridDim.x, with a bounded number of
+// polls.  Both are called by every thread of the block.
+__device__ void grid_arrive(unsigned long long *ctr) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        atomicAdd(ctr, 1ull);
+    }
+}
+
+__device__ bool grid_wait(unsigned long long *ctr, unsigned long long target) {
     __shared__ int s_ok;
     __syncthreads();
     if (threadIdx.x == 0) {
         int ok = 0;
-        __threadfence();
-        const unsigned long long old = atomicAdd(ctr, 1ull);
-        if (old + 1 >= target) {
-            ok = 1;
-        } else {
-            const volatile unsigned long long *v = ctr;
-            for (uint32_t it = 0; it < kBarrierPolls; ++it) {
-                if (*v >= target) {
-                    ok = 1;
-                    break;
-                }
-                if (it > 64) __nanosleep(32);
+        const volatile unsigned long long *v = ctr;
+        for (uint32_t it = 0; it < kBarrierPolls; ++it) {
+            if (*v >= target) {
+                ok = 1;
+                break;
             }
+            if (it > 64) __nanosleep(32);
         }
         __threadfence();
         s_ok = ok;
     }
     __syncthreads();
     return s_ok != 0;
+}
+
+// Shared-memory outputs of the alias chain, indexed by rank.
+struct AliasOut {
+    int *keep, *rfrom, *rstart, *rlen, *doff, *dlist;
+};
+
+// The balancing assignment in closed form, run by one warp: rank h lives on
+// lane h % 32, slot h / 32 (NS slots cover R <= 32 * NS ranks).
+template <int NS>
+__device__ __forceinline__ void alias_chain(int R, int C, const int *s_L, const AliasOut &o) {
+    const int lane = threadIdx.x & 31;
+    int Lv[NS], D[NS], X[NS], Pin[NS], Qin[NS], Pex[NS], Qex[NS];
+    int carryP = 0, carryQ = 0;
+#pragma unroll
+    for (int sl = 0; sl < NS; ++sl) {
+        const int h = lane + 32 * sl;
+        Lv[sl] = h < R ? s_L[h] : C;
+        D[sl] = max(C - Lv[sl], 0);
+        X[sl] = max(Lv[sl] - C, 0);
+        Pin[sl] = warp_incl_scan(D[sl]) + carryP;
+        Qin[sl] = warp_incl_scan(X[sl]) + carryQ;
+        carryP = __shfl_sync(0xffffffffu, Pin[sl], 31);
+        carryQ = __shfl_sync(0xffffffffu, Qin[sl], 31);
+        Pex[sl] = Pin[sl] - D[sl];
+        Qex[sl] = Qin[sl] - X[sl];
+    }
+    unsigned smallb[NS], largeb[NS];
+#pragma unroll
+    for (int sl = 0; sl < NS; ++sl) {
+        smallb[sl] = __ballot_sync(0xffffffffu, D[sl] > 0);
+        largeb[sl] = __ballot_sync(0xffffffffu, X[sl] > 0);
+    }
+    int donor[NS], off[NS], amt[NS];
+#pragma unroll
+    for (int sl = 0; sl < NS; ++sl) donor[sl] = -1, off[sl] = 0, amt[sl] = 0;
+    // small ranks: the large rank whose excess interval holds Pex
+#pragma unroll
+    for (int sl2 = 0; sl2 < NS; ++sl2)
+        for (unsigned m = largeb[sl2]; m; m &= m - 1) {
+            const int l = __ffs(m) - 1;
+            const int qe = __shfl_sync(0xffffffffu, Qex[sl2], l);
+            const int qi = __shfl_sync(0xffffffffu, Qin[sl2], l);
+#pragma unroll
+            for (int sl = 0; sl < NS; ++sl)
+                if (D[sl] > 0 && qe <= Pex[sl] && Pex[sl] < qi) {
+                    donor[sl] = l + 32 * sl2;
+                    off[sl] = Pex[sl] - qe;
+                    amt[sl] = D[sl];
+                }
+        }
+    // drained large ranks: a small demand interval strictly holds Qin; the
+    // rest comes from the next large rank
+#pragma unroll
+    for (int sl2 = 0; sl2 < NS; ++sl2)
+        for (unsigned m = smallb[sl2]; m; m &= m - 1) {
+            const int s = __ffs(m) - 1;
+            const int pe = __shfl_sync(0xffffffffu, Pex[sl2], s);
+            const int pi = __shfl_sync(0xffffffffu, Pin[sl2], s);
+#pragma unroll
+            for (int sl = 0; sl < NS; ++sl)
+                if (X[sl] > 0 && pe < Qin[sl] && Qin[sl] < pi) {
+                    int nxt = -1;
+                    const unsigned above_mask = ~((2u << lane) - 1u);  // lanes above this one (0 for lane 31)
+#pragma unroll
+                    for (int t = NS - 1; t >= sl; --t) {
+                        const unsigned cand = t == sl ? (largeb[t] & above_mask) : largeb[t];
+                        if (cand) nxt = 32 * t + __ffs(cand) - 1;
+                    }
+                    donor[sl] = nxt;
+                    off[sl] = 0;
+                    amt[sl] = pi - Qin[sl];
+                }
+        }
+    int keep[NS], start[NS];
+#pragma unroll
+    for (int sl = 0; sl < NS; ++sl) keep[sl] = D[sl] > 0 ? Lv[sl] : C - (X[sl] > 0 ? amt[sl] : 0);
+#pragma unroll
+    for (int sl = 0; sl < NS; ++sl) {
+        const int dl = donor[sl] < 0 ? 0 : donor[sl];
+        int kd = 0;
+#pragma unroll
+        for (int t = 0; t < NS; ++t) {
+            const int k = __shfl_sync(0xffffffffu, keep[t], dl & 31);
+            if ((dl >> 5) == t) kd = k;
+        }
+        start[sl] = donor[sl] < 0 ? 0 : kd + off[sl];
+    }
+    PLAN_TRACE(9);
+    // recipients of each donor in increasing start order
+    int pos[NS], cnt[NS];
+#pragma unroll
+    for (int sl = 0; sl < NS; ++sl) pos[sl] = 0, cnt[sl] = 0;
+#pragma unroll
+    for (int sl2 = 0; sl2 < NS; ++sl2) {
+        const unsigned rb = __ballot_sync(0xffffffffu, donor[sl2] >= 0);
+        for (unsigned m = rb; m; m &= m - 1) {
+            const int s = __ffs(m) - 1;
+            const int dn = __shfl_sync(0xffffffffu, donor[sl2], s);
+            const int st = __shfl_sync(0xffffffffu, start[sl2], s);
+#pragma unroll
+            for (int sl = 0; sl < NS; ++sl) {
+                if (donor[sl] == dn && st < start[sl]) ++pos[sl];
+                if (dn == lane + 32 * sl) ++cnt[sl];
+            }
+        }
+    }
+    int doff[NS], carry = 0;
+#pragma unroll
+    for (int sl = 0; sl < NS; ++sl) {
+        const int incl = warp_incl_scan(cnt[sl]) + carry;
+        carry = __shfl_sync(0xffffffffu, incl, 31);
+        doff[sl] = incl - cnt[sl];
+    }
+#pragma unroll
+    for (int sl = 0; sl < NS; ++sl) {
+        const int h = lane + 32 * sl;
+        if (h < R) {
+            o.keep[h] = keep[sl];
+            o.rfrom[h] = donor[sl];
+            o.rstart[h] = start[sl];
+            o.rlen[h] = amt[sl];
+            o.doff[h] = doff[sl];
+        }
+        if (h == R) o.doff[R] = doff[sl];
+    }
+    if (R == 32 * NS && lane == 0) o.doff[R] = carry;
+    __syncwarp();
+#pragma unroll
+    for (int sl = 0; sl < NS; ++sl) {
+        const int h = lane + 32 * sl;
+        if (h < R && donor[sl] >= 0) o.dlist[o.doff[donor[sl]] + pos[sl]] = h;
+    }
 }
 
 // ---- the planner kernel ----------------------------------------------------
@@ -155,10 +295,17 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
 
     uint8_t *region1 = smem;
     uint16_t *ent_e = reinterpret_cast<uint16_t *>(smem + region1_bytes(d));
-    int32_t *ent_rank = reinterpret_cast<int32_t *>(reinterpret_cast<uint8_t *>(ent_e) +
-                                                    align256(sizeof(uint16_t) * (size_t)d.ct * K));
+    uint16_t *ent_rank = reinterpret_cast<uint16_t *>(reinterpret_cast<uint8_t *>(ent_e) +
+                                                      align256(sizeof(uint16_t) * (size_t)d.ct * K));
     int32_t *tpe_s = reinterpret_cast<int32_t *>(smem + region1_bytes(d) + ent_bytes(d));  // [R][E], block 0
     const bool checker = blockIdx.x == 0 && a.tpe != nullptr;
+    const int CW = d.cw;
+    uint16_t *wcnt = reinterpret_cast<uint16_t *>(region1);                       // [CW][E]
+    uint32_t *wmask = reinterpret_cast<uint32_t *>(region1 + counts_bytes(d));    // [CW][E]
+    for (int i = tid; i < CW * E; i += kPlanThreads) {
+        wcnt[i] = 0;
+        wmask[i] = 0u;
+    }
     // the plan's status starts at 0 (block 0, before the grid barrier); every
     // later update is an atomicOr, so no error bit can be overwritten
     if (blockIdx.x == 0 && tid == 0) *a.plan.status = 0;
@@ -181,14 +328,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
     const int64_t base = ((int64_t)r * d.S + t0) * K;
 
     // ---------------- A. count ----------------
-    const int CW = d.cw;
-    uint16_t *wcnt = reinterpret_cast<uint16_t *>(region1);                       // [CW][E]
-    uint32_t *wmask = reinterpret_cast<uint32_t *>(region1 + counts_bytes(d));    // [CW][E]
     int bad = 0;
-    for (int i = tid; i < CW * E; i += kPlanThreads) {
-        wcnt[i] = 0;
-        wmask[i] = 0u;
-    }
     for (int i = tid; i < n_ent; i += kPlanThreads) {
         const int e = __ldg(a.topk + base + i);
         const bool good = e >= 0 && e < E;
@@ -229,7 +369,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
             __syncwarp();
             if (good && before == 0) mine[e] = (uint16_t)(prior + __popc(peers));
             __syncwarp();
-            if (i < w1) ent_rank[i] = prior + before;
+            if (i < w1) ent_rank[i] = (uint16_t)(prior + before);
         }
     }
     if (!whole_tokens) {  // tokens straddle runs: check duplicates token by token
@@ -261,19 +401,19 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
         __stcg(hrow + e, run);
         if (run) atomicAdd(crow + e, run);
     }
-    __syncthreads();
-    PLAN_TRACE(8);
-    for (int i = tid; i < n_ent; i += kPlanThreads) {
-        const int e = ent_e[i];
-        if (e != 0xFFFF) ent_rank[i] += wcnt[(i >> lg_run) * E + e];
-    }
     bad = __reduce_or_sync(0xffffffffu, bad);
     if (lane == 0 && bad) atomicOr(&s_bad, bad);
     __syncthreads();
     if (tid == 0 && s_bad) atomicOr(a.ws.status + parity, s_bad);
-
+    PLAN_TRACE(8);
+    grid_arrive(a.ws.arrive);
+    // while the other blocks arrive: each pick's rank inside the chunk
+    for (int i = tid; i < n_ent; i += kPlanThreads) {
+        const int e = ent_e[i];
+        if (e != 0xFFFF) ent_rank[i] = (uint16_t)(ent_rank[i] + wcnt[(i >> lg_run) * E + e]);
+    }
     PLAN_TRACE(5);
-    if (!grid_barrier(a.ws.arrive, (call + 1) * gridDim.x)) {
+    if (!grid_wait(a.ws.arrive, (call + 1) * gridDim.x)) {
         if (tid == 0) atomicOr(a.plan.status, MOONEP_STATUS_TIMEOUT);
         return;
     }
@@ -291,19 +431,26 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
     }
 
     // ---------------- B. layout (every block) ----------------
+    // T and pre are rewritten, once the outputs no longer need them, into the
+    // dst base and the rank limit of each expert's kept picks in this chunk
     int32_t *T = reinterpret_cast<int32_t *>(region1);  // [E] picks per expert
     int32_t *pre = T + E;               // [E] picks of each expert in histogram rows before this block's
     int32_t *es = pre + E;              // [E] start of each expert inside its group sequence
     int32_t *nhome = es + E;            // [E] kept picks of expert e on its home rank
-    int32_t *homeincl = nhome + E;      // [E] inclusive padded running sum over the home rows of e's rank
-    int32_t *homestart = homeincl + E;  // [E] first slot of home row e; later: dst base of kept picks
-    int32_t *nrecv = homestart + E;     // [R*G] picks of the j-th donor-group expert received by rank s; later: dst base
-    int32_t *ovfincl = nrecv + E;       // [R*G] inclusive padded running sum over overflow rows; later: end of range
+    // [E] first the inclusive padded running sum over the home rows of e's
+    // rank, then the dst base of a kept pick of e (dst = kbase[e] + position)
+    int32_t *kbase = nhome + E;
+    int32_t *nrecv = kbase + E;         // [R*G] picks of the j-th donor-group expert received by rank s
+    int32_t *ovfincl = nrecv + E;       // [R*G] inclusive padded running sum over the overflow rows
     int32_t *recvstart = ovfincl + E;   // [R*G] first slot of the row holding that received expert
-    int32_t *slotincl = recvstart + E;  // [R*B] inclusive padded running sum over the slot rows
-    int32_t *slotj = slotincl + R * B;  // [R*B] donor-group index of the expert in slot b
-    int16_t *qidx = reinterpret_cast<int16_t *>(slotj + R * B);  // [R*G] received-expert index, -1 none
-    int16_t *edon = qidx + E;           // [E] first recipient (in the donor's list) overlapping e's run
+    int32_t *ebase = recvstart + E;     // [E] dst base of e's donated picks taken by its first recipient
+    int32_t *eend = ebase + E;          // [E] end of that recipient's range
+    int32_t *ebase2 = eend + E;         // [E] the same for the second recipient (fast2 only)
+    int32_t *eend2 = ebase2 + E;        // [E]
+    int32_t *slotincl = eend + E + (d.fast2 ? 2 * E : 0);  // [R*B] inclusive padded running sum over the slot rows
+    int16_t *qidx = reinterpret_cast<int16_t *>(slotincl + R * B);  // [R*G] received-expert index, -1 none
+    int16_t *slotj = qidx + E;          // [R*B] donor-group index of the expert in slot b
+
     __shared__ int s_L[MOONEP_MAX_R], s_keep[MOONEP_MAX_R];
     __shared__ int s_rfrom[MOONEP_MAX_R], s_rstart[MOONEP_MAX_R], s_rlen[MOONEP_MAX_R];
     __shared__ int s_dlist[MOONEP_MAX_R], s_doff[MOONEP_MAX_R + 1];
@@ -324,35 +471,34 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
     {
         const int32_t *cnt = a.ws.cnt + (size_t)parity * R * E;
         const int32_t *mine_rows = a.ws.hist + (int64_t)r * d.nch * E;
+        // rows q < R are the per-rank counts, rows R <= q < R + c this rank's
+        // earlier chunk histograms; 16 loads in flight per batch
+        const int nrows = R + c;
         for (int e = tid; e < E; e += kPlanThreads) {
             int tot = 0, mypre = 0, myv = 0;
-            for (int r0 = 0; r0 < R; r0 += 8) {
-                int v[8];
+            for (int q0 = 0; q0 < nrows; q0 += 16) {
+                int v[16];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int rr = r0 + u;
-                    v[u] = rr < R ? ld_cg(cnt + (int64_t)rr * E + e) : 0;
+                for (int u = 0; u < 16; ++u) {
+                    const int q = q0 + u;
+                    const int32_t *src = q < R ? cnt + (int64_t)q * E + e : mine_rows + (int64_t)(q - R) * E + e;
+                    v[u] = q < nrows ? ld_cg(src) : 0;
                 }
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int rr = r0 + u;
-                    if (rr < R) {
+                for (int u = 0; u < 16; ++u) {
+                    const int q = q0 + u;
+                    if (q < R) {
                         tot += v[u];
-                        if (rr < r) mypre += v[u];
-                        if (rr == r) myv = v[u];
+                        if (q < r) mypre += v[u];
+                        if (q == r) myv = v[u];
                         if (checker) {
-                            const int t = tpe_in_smem(d) ? tpe_s[rr * E + e] : __ldg(a.tpe + (int64_t)rr * E + e);
+                            const int t = tpe_in_smem(d) ? tpe_s[q * E + e] : __ldg(a.tpe + (int64_t)q * E + e);
                             if (t != v[u]) mismatch = true;
                         }
+                    } else {
+                        mypre += v[u];  // 0 past the last row
                     }
                 }
-            }
-            for (int c0 = 0; c0 < c; c0 += 8) {
-                int v[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) v[u] = c0 + u < c ? ld_cg(mine_rows + (int64_t)(c0 + u) * E + e) : 0;
-#pragma unroll
-                for (int u = 0; u < 8; ++u) mypre += v[u];
             }
             T[e] = tot;
             pre[e] = mypre;
@@ -396,114 +542,11 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
     // donor's kept count plus its distance from the donor's excess start.
     // This equals the queue-driven chain step for step.
     if (w == 0) {
-        const int C = d.S * K;
-        int Lv[2], D[2], X[2], Pin[2], Qin[2], Pex[2], Qex[2];
-        int carryP = 0, carryQ = 0;
-#pragma unroll
-        for (int sl = 0; sl < 2; ++sl) {
-            const int h = lane + 32 * sl;
-            Lv[sl] = h < R ? s_L[h] : C;
-            D[sl] = max(C - Lv[sl], 0);
-            X[sl] = max(Lv[sl] - C, 0);
-            Pin[sl] = warp_incl_scan(D[sl]) + carryP;
-            Qin[sl] = warp_incl_scan(X[sl]) + carryQ;
-            carryP = __shfl_sync(0xffffffffu, Pin[sl], 31);
-            carryQ = __shfl_sync(0xffffffffu, Qin[sl], 31);
-            Pex[sl] = Pin[sl] - D[sl];
-            Qex[sl] = Qin[sl] - X[sl];
-        }
-        unsigned smallb[2], largeb[2];
-#pragma unroll
-        for (int sl = 0; sl < 2; ++sl) {
-            smallb[sl] = __ballot_sync(0xffffffffu, D[sl] > 0);
-            largeb[sl] = __ballot_sync(0xffffffffu, X[sl] > 0);
-        }
-        int donor[2] = {-1, -1}, off[2] = {0, 0}, amt[2] = {0, 0};
-        // small ranks: the large rank whose excess interval holds Pex
-#pragma unroll
-        for (int sl2 = 0; sl2 < 2; ++sl2)
-            for (unsigned m = largeb[sl2]; m; m &= m - 1) {
-                const int l = __ffs(m) - 1;
-                const int qe = __shfl_sync(0xffffffffu, Qex[sl2], l);
-                const int qi = __shfl_sync(0xffffffffu, Qin[sl2], l);
-#pragma unroll
-                for (int sl = 0; sl < 2; ++sl)
-                    if (D[sl] > 0 && qe <= Pex[sl] && Pex[sl] < qi) {
-                        donor[sl] = l + 32 * sl2;
-                        off[sl] = Pex[sl] - qe;
-                        amt[sl] = D[sl];
-                    }
-            }
-        // drained large ranks: a small demand interval strictly holds Qin
-#pragma unroll
-        for (int sl2 = 0; sl2 < 2; ++sl2)
-            for (unsigned m = smallb[sl2]; m; m &= m - 1) {
-                const int s = __ffs(m) - 1;
-                const int pe = __shfl_sync(0xffffffffu, Pex[sl2], s);
-                const int pi = __shfl_sync(0xffffffffu, Pin[sl2], s);
-#pragma unroll
-                for (int sl = 0; sl < 2; ++sl)
-                    if (X[sl] > 0 && pe < Qin[sl] && Qin[sl] < pi) {
-                        // the next large rank after this one
-                        const unsigned above = sl == 0 ? (largeb[0] & ~((2u << lane) - 1u)) : 0u;
-                        const unsigned above1 = sl == 1 ? (largeb[1] & ~((2u << lane) - 1u)) : largeb[1];
-                        donor[sl] = above ? __ffs(above) - 1 : 32 + __ffs(above1) - 1;
-                        off[sl] = 0;
-                        amt[sl] = pi - Qin[sl];
-                    }
-            }
-        int keep[2], start[2];
-#pragma unroll
-        for (int sl = 0; sl < 2; ++sl) keep[sl] = D[sl] > 0 ? Lv[sl] : C - (X[sl] > 0 ? amt[sl] : 0);
-#pragma unroll
-        for (int sl = 0; sl < 2; ++sl) {
-            const int dl = donor[sl] < 0 ? 0 : donor[sl];
-            const int k0 = __shfl_sync(0xffffffffu, keep[0], dl & 31);
-            const int k1 = __shfl_sync(0xffffffffu, keep[1], dl & 31);
-            start[sl] = donor[sl] < 0 ? 0 : (dl < 32 ? k0 : k1) + off[sl];
-        }
-        // recipients of each donor in increasing start order
-        int pos[2] = {0, 0}, cnt[2] = {0, 0};
-#pragma unroll
-        for (int sl2 = 0; sl2 < 2; ++sl2) {
-            const unsigned rb = __ballot_sync(0xffffffffu, donor[sl2] >= 0);
-            for (unsigned m = rb; m; m &= m - 1) {
-                const int s = __ffs(m) - 1;
-                const int dn = __shfl_sync(0xffffffffu, donor[sl2], s);
-                const int st = __shfl_sync(0xffffffffu, start[sl2], s);
-#pragma unroll
-                for (int sl = 0; sl < 2; ++sl) {
-                    if (donor[sl] == dn && st < start[sl]) ++pos[sl];
-                    if (dn == lane + 32 * sl) ++cnt[sl];
-                }
-            }
-        }
-        int doff[2], carry = 0;
-#pragma unroll
-        for (int sl = 0; sl < 2; ++sl) {
-            const int incl = warp_incl_scan(cnt[sl]) + carry;
-            carry = __shfl_sync(0xffffffffu, incl, 31);
-            doff[sl] = incl - cnt[sl];
-        }
-#pragma unroll
-        for (int sl = 0; sl < 2; ++sl) {
-            const int h = lane + 32 * sl;
-            if (h < R) {
-                s_keep[h] = keep[sl];
-                s_rfrom[h] = donor[sl];
-                s_rstart[h] = start[sl];
-                s_rlen[h] = amt[sl];
-                s_doff[h] = doff[sl];
-            }
-            if (h == R) s_doff[R] = doff[sl];
-        }
-        if (R == 64 && lane == 0) s_doff[R] = carry;
-        __syncwarp();
-#pragma unroll
-        for (int sl = 0; sl < 2; ++sl) {
-            const int h = lane + 32 * sl;
-            if (h < R && donor[sl] >= 0) s_dlist[s_doff[donor[sl]] + pos[sl]] = h;
-        }
+        AliasOut o{s_keep, s_rfrom, s_rstart, s_rlen, s_doff, s_dlist};
+        if (R <= 32)
+            alias_chain<1>(R, d.S * K, s_L, o);
+        else
+            alias_chain<2>(R, d.S * K, s_L, o);
     }
     if (w == 1 && blockIdx.x == 0) {
         int mxw = lane < kPlanWarps ? s_wmax[lane] : 0;
@@ -530,23 +573,6 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
     }
     __syncthreads();
     PLAN_TRACE(11);
-    // first recipient, in the donor's list, whose range overlaps expert e's run
-    for (int e = tid; e < E; e += kPlanThreads) {
-        const int h = e / G;
-        const int lo = max(es[e], s_keep[h]), hi = es[e] + T[e];
-        int first = -1;
-        if (lo < hi)
-            for (int k = s_doff[h]; k < s_doff[h + 1]; ++k) {
-                const int s = s_dlist[k];
-                if (s_rstart[s] + s_rlen[s] > lo) {
-                    first = k;
-                    break;
-                }
-            }
-        edon[e] = (int16_t)first;
-    }
-    PLAN_TRACE(12);
-
     // compact row table of every rank (one warp per rank)
     for (int s = w; s < R; s += kPlanWarps) {
         const int keep_s = s_keep[s];
@@ -559,7 +585,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
             const int incl = warp_incl_scan(pad_to(n, tp)) + carry;
             if (j < G) {
                 nhome[e] = n;
-                homeincl[e] = incl;
+                kbase[e] = incl;  // home-row running sum for now
             }
             carry = __shfl_sync(0xffffffffu, incl, 31);
         }
@@ -583,7 +609,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
                     ovfincl[s * G + j] = oincl;
                 }
                 if (is_slot) {
-                    slotj[s * B + q] = j;
+                    slotj[s * B + q] = (int16_t)j;
                     slotincl[s * B + q] = sincl;
                 }
                 nq += __popc(has);
@@ -593,7 +619,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
         }
         const int nslot = min(nq, B);
         for (int b = nslot + lane; b < B; b += 32) {
-            slotj[s * B + b] = -1;
+            slotj[s * B + b] = (int16_t)-1;
             slotincl[s * B + b] = scarry;
         }
         if (lane == 0) {
@@ -608,15 +634,36 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
         const int off_home = (h >= 0 && h < s) ? ocarry : 0;
         const int off_ovf = (h > s) ? carry : 0;
         const int off_slot = carry + ocarry;
+        // this rank's place in its donor's list of recipients, and the
+        // recipient just before it (whose range ends where this one starts)
+        int prev = -1;
+        if (h >= 0 && d.fast2)
+            for (int k = s_doff[h]; k < s_doff[h + 1]; ++k)
+                if (s_dlist[k] == s) prev = k > s_doff[h] ? s_dlist[k - 1] : -1;
         for (int j = lane; j < G; j += 32) {
             const int e = s * G + j;
-            homestart[e] = off_home + homeincl[e] - pad_to(nhome[e], tp);
+            kbase[e] = s * d.nvs + off_home + kbase[e] - pad_to(nhome[e], tp) - es[e];
             if (h >= 0) {
                 const int q = qidx[s * G + j];
                 const int p = pad_to(nrecv[s * G + j], tp);
-                recvstart[s * G + j] = q < 0 ? -1
-                                       : q < B ? off_slot + slotincl[s * B + q] - p
-                                               : off_ovf + ovfincl[s * G + j] - p;
+                const int st = q < 0 ? -1
+                               : q < B ? off_slot + slotincl[s * B + q] - p
+                                       : off_ovf + ovfincl[s * G + j] - p;
+                recvstart[s * G + j] = st;
+                // fast-path bases of expert eh's donated part: set by the
+                // recipient whose range holds its start (first), and by the
+                // recipient right after that one (second)
+                const int eh = h * G + j;
+                const int lo = max(es[eh], s_keep[h]);
+                const int a0 = s_rstart[s], a1 = a0 + s_rlen[s];
+                if (q >= 0 && a0 <= lo && lo < a1) {
+                    ebase[eh] = s * d.nvs + st - max(es[eh], a0);
+                    eend[eh] = a1;
+                } else if (d.fast2 && q >= 0 && prev >= 0 && s_rstart[prev] <= lo &&
+                           lo < s_rstart[prev] + s_rlen[prev]) {
+                    ebase2[eh] = s * d.nvs + st - a0;
+                    eend2[eh] = a1;
+                }
             }
         }
     }
@@ -627,8 +674,15 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
     auto upto = [&](int s, int i) -> int {
         int v = 0;
         const int hs = s * G;
-        if (i >= hs) v += i < hs + G ? homeincl[i] : s_hsize[s];
         const int h = s_rfrom[s];
+        if (i >= hs) {
+            if (i < hs + G) {  // the home-row running sum, recovered from kbase
+                const int off_home = (h >= 0 && h < s) ? s_osize[s] : 0;
+                v += kbase[i] - s * d.nvs - off_home + pad_to(nhome[i], tp) + es[i];
+            } else {
+                v += s_hsize[s];
+            }
+        }
         if (h >= 0) {
             const int hd = h * G;
             if (i >= hd) v += i < hd + G ? ovfincl[s * G + (i - hd)] : s_osize[s];
@@ -660,57 +714,65 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
         }
     }
     {
-        const int64_t total = (int64_t)R * NR;
-        const int64_t per = (total + gridDim.x - 1) / gridDim.x;
-        const int64_t i0 = (int64_t)blockIdx.x * per, i1 = min(total, i0 + per);
-        for (int64_t idx = i0 + tid; idx < i1; idx += kPlanThreads) {
-            const int s = (int)(idx / NR), i = (int)(idx - (int64_t)s * NR);
+        // R*(E+B) and R*B are far below 2^31 under the config limits
+        const int total = R * NR;
+        const int per = (total + (int)gridDim.x - 1) / (int)gridDim.x;
+        const int i0 = (int)blockIdx.x * per, i1 = min(total, i0 + per);
+        for (int idx = i0 + tid; idx < i1; idx += kPlanThreads) {
+            const int s = idx / NR, i = idx - s * NR;
             a.plan.cu_seqlens[idx] = upto(s, i);
             a.plan.row_counts[idx] = count_of(s, i);
         }
-        const int64_t tb = (int64_t)R * B;
-        const int64_t perb = (tb + gridDim.x - 1) / gridDim.x;
-        const int64_t b0 = (int64_t)blockIdx.x * perb, b1 = min(tb, b0 + perb);
-        for (int64_t idx = b0 + tid; idx < b1; idx += kPlanThreads) {
-            const int s = (int)(idx / B), b = (int)(idx - (int64_t)s * B);
+        const int tb = R * B;
+        const int perb = (tb + (int)gridDim.x - 1) / (int)gridDim.x;
+        const int b0 = (int)blockIdx.x * perb, b1 = min(tb, b0 + perb);
+        for (int idx = b0 + tid; idx < b1; idx += kPlanThreads) {
+            const int s = idx / B, b = idx - s * B;
             a.plan.slot_expert[idx] = b < s_nslot[s] ? s_rfrom[s] * G + slotj[idx] : -1;
         }
     }
-    __syncthreads();
     PLAN_TRACE(13);
-    // per-expert dst bases: kept picks land at kbase + g; donated picks of the
-    // first recipient overlapping the expert land at ebase + g while g < eend
-    int32_t *kbase = homestart, *ebase = nrecv, *eend = ovfincl;
+    // Fold this block's offset of each expert (its start in the group
+    // sequence plus the picks of earlier chunks) into the bases and limits,
+    // so a pick of rank rk inside the chunk needs only rk: its position in
+    // the group sequence is g = off + rk.  Nothing above reads the arrays
+    // rewritten here (T, pre, ebase, eend, ebase2, eend2).
     for (int e = tid; e < E; e += kPlanThreads) {
-        const int h = e / G;
-        kbase[e] = h * d.nvs + homestart[e] - es[e];
-        const int k = edon[e];
-        if (k >= 0) {
-            const int s = s_dlist[k];
-            ebase[e] = s * d.nvs + recvstart[s * G + (e - h * G)] - max(es[e], s_rstart[s]);
-            eend[e] = s_rstart[s] + s_rlen[s];
-        } else {
-            ebase[e] = 0;
-            eend[e] = 0;
+        const int t = T[e];
+        const int off = es[e] + pre[e];
+        const int keep = s_keep[e / G];
+        T[e] = kbase[e] + off;  // kept pick: dst = T[e] + rk ...
+        pre[e] = keep - off;    // ... while rk < pre[e]
+        if (es[e] + t > keep) {  // e has donated picks, so its first recipient set ebase/eend
+            const int e1 = eend[e];
+            ebase[e] += off;
+            eend[e] = e1 - off;
+            if (d.fast2 && es[e] + t > e1) {  // and they run on into a second recipient
+                ebase2[e] += off;
+                eend2[e] -= off;
+            }
         }
     }
     __syncthreads();
-    PLAN_TRACE(14);
+    PLAN_TRACE(12);
     // destination of every pick of this block's chunk
     for (int i = tid; i < n_ent; i += kPlanThreads) {
         const int e = ent_e[i];
-        const int h = e / G;
-        const int g = es[e] + pre[e] + ent_rank[i];
+        const int rk = ent_rank[i];
         int dst;
-        if (g < s_keep[h]) {
-            dst = kbase[e] + g;
-        } else if (g < eend[e]) {
-            dst = ebase[e] + g;
-        } else {  // the expert's donated run spans several recipients
+        if (rk < pre[e]) {
+            dst = T[e] + rk;
+        } else if (rk < eend[e]) {
+            dst = ebase[e] + rk;
+        } else if (d.fast2 && rk < eend2[e]) {
+            dst = ebase2[e] + rk;
+        } else {  // the expert's donated run spans three or more recipients
+            const int h = e / G;
+            const int g = rk + s_keep[h] - pre[e];
             int dest = -1;
-            for (int k = edon[e] + 1; k >= 1 && k < s_doff[h + 1]; ++k) {
+            for (int k = s_doff[h]; k < s_doff[h + 1]; ++k) {
                 const int s = s_dlist[k];
-                if (g < s_rstart[s] + s_rlen[s]) {
+                if (g >= s_rstart[s] && g < s_rstart[s] + s_rlen[s]) {
                     dest = s;
                     break;
                 }
