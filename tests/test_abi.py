@@ -77,3 +77,12 @@ def test_null_arguments_are_rejected():
     assert moonep.lib.moonep_reduce_grad(None, None, 1, None, None, 8, None) == moonep.ERR_NULL
     assert moonep.lib.moonep_destroy(None) == moonep.OK
     assert moonep.lib.moonep_nvs(None) < 0
+
+
+def test_buffer_layer_imports_and_names_status_bits():
+    from load_balancing_planner_b200 import moonep
+    from load_balancing_planner_b200.buffer import Buffer, PlanStatusError
+    e = PlanStatusError(moonep.STATUS_BAD_EXPERT | moonep.STATUS_COUNT_MISMATCH)
+    assert e.status == 5 and "outside [0, E)" in str(e) and "tokens_per_expert" in str(e)
+    for name in ("dispatch", "combine", "prefetch_weight", "reduce_grad", "destroy", "check"):
+        assert callable(getattr(Buffer, name))
