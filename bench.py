@@ -65,10 +65,18 @@ def describe(w):
 def dc_bytes(R, S, K, H):
     """Algorithmic bytes of dispatch + combine for one layer (all R ranks):
     dispatch reads each row once and writes it K times, plus dst, w and w_nvs;
-    combine reads K rows per token and writes one, plus dst and the weights."""
+    combine reads K rows per token and writes one, plus dst, the slot weights
+    and the gathered weights it writes back in token order."""
     disp = R * (S * H * 2 + S * K * H * 2 + 3 * S * K * 4)
-    comb = R * (S * K * H * 2 + S * H * 2 + 2 * S * K * 4)
+    comb = R * (S * K * H * 2 + S * H * 2 + 3 * S * K * 4)
     return disp, comb
+
+
+# kernels one step launches: plan_kernel, one dispatch kernel, combine_kernel
+KERNELS_PER_STEP = 3
+# the pages' own benchmark also reports maxvio 10 and 20 (outside the sweep
+# that `value` covers); timed after the run on the training shape
+PAGES_POINTS = (10.0, 20.0)
 
 
 def recorded_traffic(kernel):
@@ -268,6 +276,46 @@ def run_ours(args, world, rank, local):
     total_ms = t_start.elapsed_time(t_end)
     total_ms_max = max_over_ranks(total_ms, world)
 
+    # the planner alone, launched back to back (outside the timed region)
+    b0 = torch.cuda.Event(enable_timing=True)
+    b1 = torch.cuda.Event(enable_timing=True)
+    nb = 200
+    b0.record(stream)
+    for i in range(nb):
+        r = routes[i % npts]
+        moonep.moonep_plan(h, r["topk"], r["tpe"], plan)
+    b1.record(stream)
+    torch.cuda.synchronize()
+    plan_b2b_us = b0.elapsed_time(b1) * 1e3 / nb
+
+    # The same steps without planning, each routing's plan computed ahead:
+    # the planner's cost per layer is the difference in step time.  Both
+    # loops record the same four events per step.
+    saved = []
+    for r in routes:
+        saved.append(moonep.moonep_plan(h, r["topk"], r["tpe"], moonep.Plan(h, dev)))
+
+    def step_saved(i, ev=None):
+        p = saved[i % npts]
+        if ev:
+            ev[0].record(stream)
+            ev[1].record(stream)
+        moonep.moonep_dispatch(h, p, hidden, weights, buf, wn)
+        if ev:
+            ev[2].record(stream)
+        moonep.moonep_combine(h, p, buf, wn, out, gw)
+        if ev:
+            ev[3].record(stream)
+
+    for i in range(args.warmup):
+        step_saved(i)
+    evs2 = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    for i in range(args.steps):
+        step_saved(i, evs2[i])
+    torch.cuda.synchronize()
+    with_ms = [e[0].elapsed_time(e[3]) for e in evs]
+    without_ms = [e[0].elapsed_time(e[3]) for e in evs2]
+
     plan_ms = [e[0].elapsed_time(e[1]) for e in evs]
     disp_ms = [e[1].elapsed_time(e[2]) for e in evs]
     comb_ms = [e[2].elapsed_time(e[3]) for e in evs]
@@ -283,7 +331,10 @@ def run_ours(args, world, rank, local):
         dc = statistics.median([disp_ms[i] + comb_ms[i] for i in idx])
         gbs = (db + cb) / (dc * 1e-3) / 1e9
         sweep[f"{r['target']:g}"] = dict(
-            realised_maxvio=round(r["realised"], 4), planner_us=round(statistics.median([plan_ms[i] for i in idx]) * 1e3, 2),
+            realised_maxvio=round(r["realised"], 4),
+            planner_us=round((statistics.median([with_ms[i] for i in idx]) -
+                              statistics.median([without_ms[i] for i in idx])) * 1e3, 2),
+            planner_us_event_bracketed=round(statistics.mean([plan_ms[i] for i in idx]) * 1e3, 2),
             dispatch_us=round(statistics.median([disp_ms[i] for i in idx]) * 1e3, 1),
             combine_us=round(statistics.median([comb_ms[i] for i in idx]) * 1e3, 1),
             dc_gbs=round(gbs, 1), dc_frac_measured=round(gbs / peak, 4), dc_frac_8tbs=round(gbs / NOMINAL_HBM_GBS, 4))
@@ -310,7 +361,13 @@ def run_ours(args, world, rank, local):
                    "l2": "inputs larger than L2 (hidden rows 470 MB, dispatch buffer 4.7 GB per layer)"
                    if args.config == "train" else "inputs larger than L2",
                    "step": "plan + dispatch + combine of one layer; combine reads the dispatch buffer"},
-        "planner_us": round(statistics.median(plan_ms) * 1e3, 2),
+        # planner per layer: median step time with planning minus median
+        # step time with saved plans, per routing, averaged over the sweep;
+        # also the planner between two CUDA events in each step (those come
+        # in ~2 us steps), and launched back to back alone
+        "planner_us": round(statistics.mean(v["planner_us"] for v in sweep.values()), 2),
+        "planner_us_event_bracketed": round(statistics.mean(plan_ms) * 1e3, 2),
+        "planner_us_back_to_back": round(plan_b2b_us, 2),
         "dispatch_gbs": round(db / (statistics.median(disp_ms) * 1e-3) / 1e9, 1),
         "combine_gbs": round(cb / (statistics.median(comb_ms) * 1e-3) / 1e9, 1),
         "dc_frac_measured_min": round(min(v["dc_frac_measured"] for v in sweep.values()), 4),
@@ -318,16 +375,55 @@ def run_ours(args, world, rank, local):
         "spread_vs_maxvio": round(spread, 4) if spread is not None else None,
         "sweep": sweep,
         "roofline": roofline,
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": KERNELS_PER_STEP * args.steps,
         "clocks": clk,
     }
 
     if not args.no_legs:
         result["legs"] = run_legs(args, dev, world)
+        if args.config == "train":
+            result["legs"]["pages_maxvio_points"] = run_pages_points(w, seed, dev, h, plan, hidden, weights,
+                                                                     buf, wn, out, gw, stream)
     if not args.no_e2e:
         result["e2e"] = run_e2e(args, h, plan, w, routes, dev, stream, world)
     h.close()
     return result, routes
+
+
+def run_pages_points(w, seed, dev, h, plan, hidden, weights, buf, wn, out, gw, stream, reps=20):
+    """plan + dispatch + combine at the maxvio 10 and 20 points of the pages'
+    benchmark, on the training shape and buffers (CUDA events, medians)."""
+    import torch
+    from load_balancing_planner_b200 import moonep
+    R, S, K, E, H = w["R"], w["S"], w["K"], w["E"], w["H"]
+    db, cb = dc_bytes(R, S, K, H)
+    pts = {}
+    for mv in PAGES_POINTS:
+        tk, real, _ = synth.routing(R, S, K, E, mv, w["profile"], seed=seed)
+        topk = torch.from_numpy(tk).to(dev)
+        tpe = torch.from_numpy(synth.local_counts(tk, E)).to(dev)
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(reps + 3)]
+        for e in evs:
+            e[0].record(stream)
+            moonep.moonep_plan(h, topk, tpe, plan)
+            e[1].record(stream)
+            moonep.moonep_dispatch(h, plan, hidden, weights, buf, wn)
+            e[2].record(stream)
+            moonep.moonep_combine(h, plan, buf, wn, out, gw)
+            e[3].record(stream)
+        torch.cuda.synchronize()
+        if moonep.moonep_read_status(plan) != 0:
+            raise RuntimeError(f"plan status at maxvio {mv}")
+        evs = evs[3:]
+        dc = statistics.median([e[1].elapsed_time(e[3]) for e in evs])
+        pts[f"{mv:g}"] = dict(realised_maxvio=round(real, 4),
+                              planner_us_event_bracketed=round(
+                                  statistics.mean([e[0].elapsed_time(e[1]) for e in evs]) * 1e3, 2),
+                              dispatch_us=round(statistics.median([e[1].elapsed_time(e[2]) for e in evs]) * 1e3, 1),
+                              combine_us=round(statistics.median([e[2].elapsed_time(e[3]) for e in evs]) * 1e3, 1),
+                              dc_gbs=round((db + cb) / (dc * 1e-3) / 1e9, 1),
+                              used_slots=int((plan.slots() >= 0).sum().item()))
+    return pts
 
 
 def run_legs(args, dev, world):
@@ -400,7 +496,13 @@ def run_legs(args, dev, world):
 
 def run_e2e(args, h, plan, w, routes, dev, stream, world):
     """The same step through the C ABI from pinned host buffers: H2D of the
-    step's inputs, plan, dispatch, combine, D2H of the combined output."""
+    step's inputs, plan, dispatch, combine, D2H of the combined output.
+
+    Steps are pipelined over three streams with two buffer sets, the way a
+    data loader feeds a GPU: step i+1's inputs go up and step i-1's output
+    comes down (PCIe is full duplex) while step i computes.  Every step's
+    copies are inside the timed region, which runs from the first upload to
+    the last download."""
     import torch
     from load_balancing_planner_b200 import moonep
     R, S, K, E, H = w["R"], w["S"], w["K"], w["E"], w["H"]
@@ -409,44 +511,65 @@ def run_e2e(args, h, plan, w, routes, dev, stream, world):
     wts_h = torch.from_numpy(synth.route_weights(R, S, K, args.seed)).pin_memory()
     tks_h = [r["topk"].cpu().pin_memory() for r in routes]
     tpe_h = [r["tpe"].cpu().pin_memory() for r in routes]
-    out_h = torch.empty((R, S, H), dtype=torch.bfloat16).pin_memory()
-    hid_d = torch.empty((R, S, H), dtype=torch.bfloat16, device=dev)
-    wts_d = torch.empty((R, S, K), dtype=torch.float32, device=dev)
-    tk_d = torch.empty((R, S, K), dtype=torch.int32, device=dev)
-    tpe_d = torch.empty((R, E), dtype=torch.int32, device=dev)
+    out_h = [torch.empty((R, S, H), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    hid_d = [torch.empty((R, S, H), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    wts_d = [torch.empty((R, S, K), dtype=torch.float32, device=dev) for _ in range(2)]
+    tk_d = [torch.empty((R, S, K), dtype=torch.int32, device=dev) for _ in range(2)]
+    tpe_d = [torch.empty((R, E), dtype=torch.int32, device=dev) for _ in range(2)]
+    out = [torch.empty((R, S, H), dtype=torch.bfloat16, device=dev) for _ in range(2)]
     buf = torch.empty((R, nvs, H), dtype=torch.bfloat16, device=dev)
     wn = torch.empty((R, nvs), dtype=torch.float32, device=dev)
-    out = torch.empty((R, S, H), dtype=torch.bfloat16, device=dev)
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = {k: [torch.cuda.Event() for _ in range(2)] for k in ("up", "done", "down")}
+    used = {k: [False, False] for k in ev}
 
     def step(i):
-        j = i % len(routes)
-        hid_d.copy_(hid_h, non_blocking=True)
-        wts_d.copy_(wts_h, non_blocking=True)
-        tk_d.copy_(tks_h[j], non_blocking=True)
-        tpe_d.copy_(tpe_h[j], non_blocking=True)
-        moonep.moonep_plan(h, tk_d, tpe_d, plan)
-        moonep.moonep_dispatch(h, plan, hid_d, wts_d, buf, wn)
-        moonep.moonep_combine(h, plan, buf, wn, out, None, gather=False)
-        out_h.copy_(out, non_blocking=True)
+        j, sl = i % len(routes), i % 2
+        with torch.cuda.stream(up):
+            if used["done"][sl]:
+                up.wait_event(ev["done"][sl])  # step i-2 no longer reads these inputs
+            hid_d[sl].copy_(hid_h, non_blocking=True)
+            wts_d[sl].copy_(wts_h, non_blocking=True)
+            tk_d[sl].copy_(tks_h[j], non_blocking=True)
+            tpe_d[sl].copy_(tpe_h[j], non_blocking=True)
+            ev["up"][sl].record(up)
+        stream.wait_event(ev["up"][sl])
+        if used["down"][sl]:
+            stream.wait_event(ev["down"][sl])  # step i-2's output has left the device
+        moonep.moonep_plan(h, tk_d[sl], tpe_d[sl], plan, stream=stream)
+        moonep.moonep_dispatch(h, plan, hid_d[sl], wts_d[sl], buf, wn, stream=stream)
+        moonep.moonep_combine(h, plan, buf, wn, out[sl], None, gather=False, stream=stream)
+        ev["done"][sl].record(stream)
+        with torch.cuda.stream(down):
+            down.wait_event(ev["done"][sl])
+            out_h[sl].copy_(out[sl], non_blocking=True)
+            ev["down"][sl].record(down)
+        for k in ev:
+            used[k][sl] = True
 
-    n = max(5, min(args.steps, 2 * len(routes)))
+    n = max(6, min(args.steps, 2 * len(routes)))
     for i in range(2):
         step(i)
+    torch.cuda.synchronize()
     barrier(world)
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
     a.record(stream)
+    up.wait_stream(stream)  # the first upload starts after the start mark
     for i in range(n):
         step(i)
+    stream.wait_stream(down)  # the end mark follows the last download
     b.record(stream)
     torch.cuda.synchronize()
     barrier(world)
     ms = max_over_ranks(a.elapsed_time(b), world)
     db, cb = dc_bytes(R, S, K, H)
+    cb -= R * S * K * 4  # this combine does not gather the weights back
     h2d = hid_h.numel() * 2 + wts_h.numel() * 4 + tks_h[0].numel() * 4 + tpe_h[0].numel() * 4
     return {"value": round(aggregate_gbs(db + cb, n, world, ms), 1), "unit": "GB/s",
-            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(out_h.numel() * 2),
-            "ms_per_step": round(ms / n, 3), "steps": n}
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(out_h[0].numel() * 2),
+            "ms_per_step": round(ms / n, 3), "steps": n,
+            "pipelined": "uploads, compute and downloads of consecutive steps overlap on 3 streams"}
 
 
 # ---------------------------------------------------------------- the oracle
@@ -522,6 +645,35 @@ def run_reference(args, world, rank):
     }
 
 
+def run_planner_only(args):
+    """The planner alone on the workload's routings, back to back: a small
+    program (the routing and plan arrays only) for profiler captures."""
+    import torch
+    from load_balancing_planner_b200 import moonep
+    w = WORKLOADS[args.config]
+    R, S, K, E, B, H, tp = w["R"], w["S"], w["K"], w["E"], w["B"], w["H"], w["tp"]
+    dev = torch.device("cuda", 0)
+    routes = []
+    for mv in w["maxvio"]:
+        tk, _, _ = synth.routing(R, S, K, E, mv, w["profile"], seed=args.seed)
+        routes.append((torch.from_numpy(tk).to(dev), torch.from_numpy(synth.local_counts(tk, E)).to(dev)))
+    h = moonep.moonep_create(S, H, K, E, R, B, tp, mode=w["mode"])
+    plan = moonep.Plan(h, dev)
+    for i in range(args.warmup):
+        moonep.moonep_plan(h, *routes[i % len(routes)], plan)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for i in range(args.steps):
+        moonep.moonep_plan(h, *routes[i % len(routes)], plan)
+    b.record()
+    torch.cuda.synchronize()
+    st = moonep.moonep_read_status(plan)
+    h.close()
+    return {"planner_only": args.config, "launches": args.warmup + args.steps, "status": st,
+            "back_to_back_us": round(a.elapsed_time(b) * 1e3 / args.steps, 2)}
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -535,9 +687,15 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--traffic", type=float, default=None,
                     help="ncu DRAM bytes per launch of the dominant kernel, if measured for this build")
+    ap.add_argument("--planner-only", action="store_true",
+                    help="launch only the planner (every routing of the workload), for profiler captures; "
+                         "prints its back-to-back time, not a bench line")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.planner_only:
+        print(json.dumps(run_planner_only(args)), flush=True)
+        return
 
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))

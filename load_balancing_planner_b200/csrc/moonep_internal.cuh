@@ -13,7 +13,7 @@ namespace moonep {
 // source rank (all blocks resident), kPlanThreads threads each.
 constexpr int kPlanThreads = 1024;
 constexpr int kPlanWarps = kPlanThreads / 32;
-constexpr int kChunkTokensMin = 512;
+constexpr int kChunkTokensMin = 256;
 constexpr int kMaxDevices = 64;
 constexpr uint32_t kBarrierPolls = 1u << 22;  // each poll is an L2 round trip: ~2 s, then MOONEP_STATUS_TIMEOUT
 

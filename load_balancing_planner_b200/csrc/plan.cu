@@ -77,9 +77,10 @@ size_t plan_smem_bytes(const Dims &d) {
 // Phase timestamps for profiling builds (-DMOONEP_PLAN_TRACE); no code otherwise.
 #ifdef MOONEP_PLAN_TRACE
 __device__ unsigned long long g_plan_trace[1024][16];
-#define PLAN_TRACE(k)                                                                      \
+#define PLAN_TRACE(k) PLAN_TRACE_BY(k, 0)
+#define PLAN_TRACE_BY(k, t)                                                                \
     do {                                                                                   \
-        if (threadIdx.x == 0 && blockIdx.x < 1024) {                                       \
+        if (threadIdx.x == (t) && blockIdx.x < 1024) {                                     \
             unsigned long long t_;                                                         \
             asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                         \
             g_plan_trace[blockIdx.x][k] = t_;                                              \
@@ -91,6 +92,9 @@ extern "C" __attribute__((visibility("default"))) int moonep_plan_trace(unsigned
 #else
 #define PLAN_TRACE(k) \
     do {              \
+    } while (0)
+#define PLAN_TRACE_BY(k, t) \
+    do {                    \
     } while (0)
 #endif
 
@@ -443,8 +447,10 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
     int32_t *nrecv = kbase + E;         // [R*G] picks of the j-th donor-group expert received by rank s
     int32_t *ovfincl = nrecv + E;       // [R*G] inclusive padded running sum over the overflow rows
     int32_t *recvstart = ovfincl + E;   // [R*G] first slot of the row holding that received expert
-    int32_t *ebase = recvstart + E;     // [E] dst base of e's donated picks taken by its first recipient
-    int32_t *eend = ebase + E;          // [E] end of that recipient's range
+    // [E] e's donated picks at their first recipient: dst = ebase[e] + rk for
+    // a pick of chunk rank rk below eend[e] (both relative to this chunk)
+    int32_t *ebase = recvstart + E;
+    int32_t *eend = ebase + E;
     int32_t *ebase2 = eend + E;         // [E] the same for the second recipient (fast2 only)
     int32_t *eend2 = ebase2 + E;        // [E]
     int32_t *slotincl = eend + E + (d.fast2 ? 2 * E : 0);  // [R*B] inclusive padded running sum over the slot rows
@@ -650,19 +656,22 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
                                : q < B ? off_slot + slotincl[s * B + q] - p
                                        : off_ovf + ovfincl[s * G + j] - p;
                 recvstart[s * G + j] = st;
-                // fast-path bases of expert eh's donated part: set by the
-                // recipient whose range holds its start (first), and by the
-                // recipient right after that one (second)
+                // fast-path bases of expert eh's donated part, set by the
+                // recipient whose range holds its start (first) and by the
+                // recipient right after that one (second).  They are taken
+                // relative to this block's chunk: a pick of chunk rank rk
+                // sits at g = off + rk in the group sequence.
                 const int eh = h * G + j;
+                const int off = es[eh] + pre[eh];
                 const int lo = max(es[eh], s_keep[h]);
                 const int a0 = s_rstart[s], a1 = a0 + s_rlen[s];
                 if (q >= 0 && a0 <= lo && lo < a1) {
-                    ebase[eh] = s * d.nvs + st - max(es[eh], a0);
-                    eend[eh] = a1;
+                    ebase[eh] = s * d.nvs + st - max(es[eh], a0) + off;
+                    eend[eh] = a1 - off;
                 } else if (d.fast2 && q >= 0 && prev >= 0 && s_rstart[prev] <= lo &&
                            lo < s_rstart[prev] + s_rlen[prev]) {
-                    ebase2[eh] = s * d.nvs + st - a0;
-                    eend2[eh] = a1;
+                    ebase2[eh] = s * d.nvs + st - a0 + off;
+                    eend2[eh] = a1 - off;
                 }
             }
         }
@@ -704,21 +713,25 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
         return b < s_nslot[s] ? nrecv[s * G + slotj[s * B + b]] : 0;
     };
 
-    // ---------------- C. outputs ----------------
-    if (blockIdx.x == 0) {
-        for (int j = tid; j < R; j += kPlanThreads) {
-            a.plan.assign[4 * j + 0] = s_keep[j];
-            a.plan.assign[4 * j + 1] = s_rfrom[j];
-            a.plan.assign[4 * j + 2] = s_rstart[j];
-            a.plan.assign[4 * j + 3] = s_rlen[j];
+    // ---------------- C. outputs and dst ----------------
+    // The first `ow` warps write this block's share of the per-rank outputs
+    // (nothing below reads them) while the other warps fold the chunk
+    // offsets into the bases and write dst, after a barrier of their own.
+    const int total = R * NR;  // R*(E+B) and R*B are far below 2^31 under the config limits
+    const int per = (total + (int)gridDim.x - 1) / (int)gridDim.x;
+    const int ow = per <= 128 ? 1 : 4;
+    if (w < ow) {
+        const int ot = 32 * ow;
+        if (blockIdx.x == 0) {
+            for (int j = tid; j < R; j += ot) {
+                a.plan.assign[4 * j + 0] = s_keep[j];
+                a.plan.assign[4 * j + 1] = s_rfrom[j];
+                a.plan.assign[4 * j + 2] = s_rstart[j];
+                a.plan.assign[4 * j + 3] = s_rlen[j];
+            }
         }
-    }
-    {
-        // R*(E+B) and R*B are far below 2^31 under the config limits
-        const int total = R * NR;
-        const int per = (total + (int)gridDim.x - 1) / (int)gridDim.x;
         const int i0 = (int)blockIdx.x * per, i1 = min(total, i0 + per);
-        for (int idx = i0 + tid; idx < i1; idx += kPlanThreads) {
+        for (int idx = i0 + tid; idx < i1; idx += ot) {
             const int s = idx / NR, i = idx - s * NR;
             a.plan.cu_seqlens[idx] = upto(s, i);
             a.plan.row_counts[idx] = count_of(s, i);
@@ -726,67 +739,58 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
         const int tb = R * B;
         const int perb = (tb + (int)gridDim.x - 1) / (int)gridDim.x;
         const int b0 = (int)blockIdx.x * perb, b1 = min(tb, b0 + perb);
-        for (int idx = b0 + tid; idx < b1; idx += kPlanThreads) {
+        for (int idx = b0 + tid; idx < b1; idx += ot) {
             const int s = idx / B, b = idx - s * B;
             a.plan.slot_expert[idx] = b < s_nslot[s] ? s_rfrom[s] * G + slotj[idx] : -1;
         }
-    }
-    PLAN_TRACE(13);
-    // Fold this block's offset of each expert (its start in the group
-    // sequence plus the picks of earlier chunks) into the bases and limits,
-    // so a pick of rank rk inside the chunk needs only rk: its position in
-    // the group sequence is g = off + rk.  Nothing above reads the arrays
-    // rewritten here (T, pre, ebase, eend, ebase2, eend2).
-    for (int e = tid; e < E; e += kPlanThreads) {
-        const int t = T[e];
-        const int off = es[e] + pre[e];
-        const int keep = s_keep[e / G];
-        T[e] = kbase[e] + off;  // kept pick: dst = T[e] + rk ...
-        pre[e] = keep - off;    // ... while rk < pre[e]
-        if (es[e] + t > keep) {  // e has donated picks, so its first recipient set ebase/eend
-            const int e1 = eend[e];
-            ebase[e] += off;
-            eend[e] = e1 - off;
-            if (d.fast2 && es[e] + t > e1) {  // and they run on into a second recipient
-                ebase2[e] += off;
-                eend2[e] -= off;
-            }
+        PLAN_TRACE(13);
+    } else {
+        const int t2 = tid - 32 * ow, n2 = kPlanThreads - 32 * ow;
+        // Fold this block's offset of each expert (its start in the group
+        // sequence plus the picks of earlier chunks) into the kept-pick base
+        // and limit, so a pick of rank rk inside the chunk needs only rk: its
+        // position in the group sequence is g = off + rk.  The outputs never
+        // read the arrays rewritten here (T, pre).
+        for (int e = t2; e < E; e += n2) {
+            const int off = es[e] + pre[e];
+            T[e] = kbase[e] + off;           // kept pick: dst = T[e] + rk ...
+            pre[e] = s_keep[e / G] - off;    // ... while rk < pre[e]
         }
-    }
-    __syncthreads();
-    PLAN_TRACE(12);
-    // destination of every pick of this block's chunk
-    for (int i = tid; i < n_ent; i += kPlanThreads) {
-        const int e = ent_e[i];
-        const int rk = ent_rank[i];
-        int dst;
-        if (rk < pre[e]) {
-            dst = T[e] + rk;
-        } else if (rk < eend[e]) {
-            dst = ebase[e] + rk;
-        } else if (d.fast2 && rk < eend2[e]) {
-            dst = ebase2[e] + rk;
-        } else {  // the expert's donated run spans three or more recipients
-            const int h = e / G;
-            const int g = rk + s_keep[h] - pre[e];
-            int dest = -1;
-            for (int k = s_doff[h]; k < s_doff[h + 1]; ++k) {
-                const int s = s_dlist[k];
-                if (g >= s_rstart[s] && g < s_rstart[s] + s_rlen[s]) {
-                    dest = s;
-                    break;
+        asm volatile("bar.sync 1, %0;" ::"r"(n2) : "memory");
+        PLAN_TRACE_BY(12, 32 * ow);
+        // destination of every pick of this block's chunk
+        for (int i = t2; i < n_ent; i += n2) {
+            const int e = ent_e[i];
+            const int rk = ent_rank[i];
+            int dst;
+            if (rk < pre[e]) {
+                dst = T[e] + rk;
+            } else if (rk < eend[e]) {
+                dst = ebase[e] + rk;
+            } else if (d.fast2 && rk < eend2[e]) {
+                dst = ebase2[e] + rk;
+            } else {  // the expert's donated run spans three or more recipients
+                const int h = e / G;
+                const int g = rk + s_keep[h] - pre[e];
+                int dest = -1;
+                for (int k = s_doff[h]; k < s_doff[h + 1]; ++k) {
+                    const int s = s_dlist[k];
+                    if (g >= s_rstart[s] && g < s_rstart[s] + s_rlen[s]) {
+                        dest = s;
+                        break;
+                    }
                 }
+                const int st = dest < 0 ? -1 : recvstart[dest * G + (e - h * G)];
+                if (st < 0) {  // unreachable for a consistent layout; never write with it
+                    atomicOr(a.plan.status, MOONEP_STATUS_BAD_PLAN);
+                    continue;
+                }
+                dst = dest * d.nvs + st + (g - max(es[e], s_rstart[dest]));
             }
-            const int st = dest < 0 ? -1 : recvstart[dest * G + (e - h * G)];
-            if (st < 0) {  // unreachable for a consistent layout; never write with it
-                atomicOr(a.plan.status, MOONEP_STATUS_BAD_PLAN);
-                continue;
-            }
-            dst = dest * d.nvs + st + (g - max(es[e], s_rstart[dest]));
+            a.plan.dst[base + i] = dst;
         }
-        a.plan.dst[base + i] = dst;
+        PLAN_TRACE_BY(4, 32 * ow);
     }
-    PLAN_TRACE(4);
     if (blockIdx.x == 0) {
         __syncthreads();
         if (tid == 0 && s_mismatch) atomicOr(a.plan.status, s_mismatch);
