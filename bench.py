@@ -107,6 +107,16 @@ def peaks():
         return 6650.0, "fallback"
 
 
+def tensor_peaks():
+    """Dense bf16 TFLOP/s: (burst, sustained, kind)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["bf16_tflops"]), float(p["bf16_tflops_sustained"]), "measured"
+    except Exception:
+        return 1590.0, 1400.0, "fallback"
+
+
 # ---------------------------------------------------------------- clocks
 class Clocks:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -384,6 +394,7 @@ def run_ours(args, world, rank, local):
         if args.config == "train":
             result["legs"]["pages_maxvio_points"] = run_pages_points(w, seed, dev, h, plan, hidden, weights,
                                                                      buf, wn, out, gw, stream)
+            result["legs"]["group_gemm"] = run_group_gemm_leg(dev, seed)
     if not args.no_e2e:
         result["e2e"] = run_e2e(args, h, plan, w, routes, dev, stream, world)
     h.close()
@@ -424,6 +435,47 @@ def run_pages_points(w, seed, dev, h, plan, hidden, weights, buf, wn, out, gw, s
                               dc_gbs=round((db + cb) / (dc * 1e-3) / 1e9, 1),
                               used_slots=int((plan.slots() >= 0).sum().item()))
     return pts
+
+
+def run_group_gemm_leg(dev, seed, mv=2.0, Hp=2048, reps=10):
+    """The VM group GEMM that consumes a dispatched training layer: one
+    [H, H'] projection per plan row (home experts from W, slot rows from the
+    prefetched pool), H' = 2048, bf16 in, fp32 accumulation, bf16 out.
+    FLOPs count the real slots only (2 * R*S*K * H * H'); the kernel also
+    multiplies each row's padding up to a multiple of 128."""
+    import torch
+    from load_balancing_planner_b200 import moonep
+    w = WORKLOADS["train"]
+    R, S, K, E, B, H, tp = w["R"], w["S"], w["K"], w["E"], w["B"], w["H"], w["tp"]
+    tk, real, _ = synth.routing(R, S, K, E, mv, w["profile"], seed=seed)
+    h = moonep.moonep_create(S, H, K, E, R, B, tp)
+    plan = moonep.moonep_plan(h, torch.from_numpy(tk).to(dev), torch.from_numpy(synth.local_counts(tk, E)).to(dev))
+    x, _ = moonep.moonep_dispatch(h, plan, synth.hidden_bf16(R, S, H, seed).to(dev))
+    g = torch.Generator(device=dev).manual_seed(seed)
+    W = (torch.randn((E, H, Hp), generator=g, device=dev) * H ** -0.5).to(torch.bfloat16)
+    pool = torch.empty((R, B, H, Hp), dtype=torch.bfloat16, device=dev)
+    moonep.moonep_prefetch_weight(h, plan, [W], [pool])
+    y = torch.empty((R, h.nvs, Hp), dtype=torch.bfloat16, device=dev)
+    for _ in range(3):
+        moonep.moonep_group_gemm(h, plan, x, W, pool, y)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for a, b in evs:
+        a.record()
+        moonep.moonep_group_gemm(h, plan, x, W, pool, y)
+        b.record()
+    torch.cuda.synchronize()
+    if moonep.moonep_read_status(plan) != 0:
+        raise RuntimeError("group GEMM: plan status")
+    us = statistics.median(a.elapsed_time(b) for a, b in evs) * 1e3
+    rows_computed = int(plan.cu_seqlens[:, -1].sum().item())
+    flops = 2.0 * R * S * K * H * Hp
+    burst, sustained, kind = tensor_peaks()
+    tf = flops / (us * 1e-6) / 1e12
+    h.close()
+    return {"workload": f"train shape, plan at maxvio {mv:g}, H'={Hp}, bf16 -> fp32 accumulate -> bf16",
+            "realised_maxvio": round(real, 4), "flops": flops, "us": round(us, 1), "tflops": round(tf, 1),
+            "frac_of_bf16_burst": round(tf / burst, 4), "frac_of_bf16_sustained": round(tf / sustained, 4),
+            "peak_kind": kind, "rows_real": R * S * K, "rows_computed": rows_computed}
 
 
 def run_legs(args, dev, world):

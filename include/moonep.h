@@ -204,6 +204,31 @@ MOONEP_API int moonep_reduce_grad(moonep_handle_t h, const moonep_plan_t *plan, 
                        moonep_stream_t stream);
 
 /*
+ * The VM group GEMM that consumes a dispatched layer (README "Integration":
+ * one [E+B, H, H'] weight tensor per projection, with cu_seqlens selecting
+ * the expert row of every token segment; "Weight buffer": rows [0, E) are the
+ * home experts, rows [E, E+B) the rank's prefetch slots).  For every rank r
+ * and every row i of its plan with row_counts[r][i] > 0:
+ *   y_nvs[r, s_i : s_i + pad(n_i), :] = x_nvs[r, s_i : s_i + pad(n_i), :] @ Wi
+ * where s_i = cu_seqlens[r][i] - pad(n_i) is the row's first slot, and
+ * Wi = weights[i] for i < E (home rows, and inference overflow rows, which
+ * read the home expert), pool[r][i - E] for slot rows.  fp32 accumulation on
+ * the tensor cores, bf16 output rounded to nearest even.  Padding slots are
+ * multiplied too (their contents are unspecified); slots after a rank's last
+ * row are not written.
+ *   x_nvs   [R,NvS,H]  bf16  the dispatched buffer
+ *   weights [E,H,Hp]   bf16  the home experts
+ *   pool    [R,B,H,Hp] bf16  every rank's prefetch slots (NULL allowed if B=0)
+ *   y_nvs   [R,NvS,Hp] bf16  output
+ * Requires token_padding % 128 == 0 (a 128-row tile never spans two rows),
+ * H % 64 == 0 and Hp % 256 == 0, else MOONEP_ERR_SIZE; pointers 16-byte
+ * aligned.  A failed plan (plan->status != 0) computes nothing.
+ */
+MOONEP_API int moonep_group_gemm(moonep_handle_t h, const moonep_plan_t *plan, const void *x_nvs,
+                                 const void *weights, const void *pool, void *y_nvs, int64_t Hp,
+                                 moonep_stream_t stream);
+
+/*
  * moonep_plan without a handle and without allocating: the same plan as
  * moonep_plan for the same cfg and inputs.  (This entry point has no
  * counterpart on the pages; it exists for callers that cannot call cudaMalloc
@@ -215,7 +240,7 @@ MOONEP_API int moonep_reduce_grad(moonep_handle_t h, const moonep_plan_t *plan, 
  * device memory, part of the library image: every GPU that loads the library
  * holds it until the process exits.  A cfg whose workspace does not fit is
  * rejected with MOONEP_ERR_SIZE (the training shape R=8, S=4096, K=8, E=256
- * needs about 80 KB).  The call allocates nothing (no cudaMalloc, cudaFree or
+ * needs about 150 KB).  The call allocates nothing (no cudaMalloc, cudaFree or
  * allocating library routine); it clears the part of the array that must
  * start at zero with cudaMemsetAsync on `stream`.
  *

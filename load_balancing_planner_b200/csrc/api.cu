@@ -91,6 +91,7 @@ int prepare_device(int device) {
     if (e == cudaSuccess) e = plan_set_smem_limit((size_t)optin - plan_static_smem_bytes());
     if (e == cudaSuccess) e = weights_set_smem_limit((size_t)optin - weights_static_smem_bytes());
     if (e == cudaSuccess) e = dispatch_bulk_set_smem_limit((size_t)optin - 1024);
+    if (e == cudaSuccess) e = gemm_set_smem_limit();
     if (e != cudaSuccess) return fail_cuda(e);
     done[device] = true;
     return MOONEP_OK;
@@ -291,6 +292,18 @@ extern "C" int moonep_reduce_grad(moonep_handle_t h, const moonep_plan_t *plan, 
     if (h->d.B == 0) return MOONEP_OK;
     const cudaError_t e = launch_reduce_grad(a, h->grid_weights, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? MOONEP_OK : fail_cuda(e);
+}
+
+extern "C" int moonep_group_gemm(moonep_handle_t h, const moonep_plan_t *plan, const void *x_nvs,
+                                 const void *weights, const void *pool, void *y_nvs, int64_t Hp,
+                                 moonep_stream_t stream) {
+    if (!h || !plan || !plan->cu_seqlens || !plan->status || !x_nvs || !weights || !y_nvs) return MOONEP_ERR_NULL;
+    if (h->d.B > 0 && !pool) return MOONEP_ERR_NULL;
+    if (!aligned16(x_nvs) || !aligned16(weights) || !aligned16(y_nvs) || (pool && !aligned16(pool)))
+        return MOONEP_ERR_ALIGN;
+    const int rc = gemm_supported(h->d, Hp);
+    if (rc != MOONEP_OK) return rc;
+    return launch_group_gemm(h->d, plan, x_nvs, weights, pool, y_nvs, Hp, reinterpret_cast<cudaStream_t>(stream));
 }
 
 extern "C" int moonep_read_status(const moonep_plan_t *plan, int32_t *status, moonep_stream_t stream) {

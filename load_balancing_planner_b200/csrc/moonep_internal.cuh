@@ -87,6 +87,12 @@ cudaError_t launch_prefetch(const WeightArgs &a, int grid, cudaStream_t st);
 cudaError_t launch_reduce_grad(const WeightArgs &a, int grid, cudaStream_t st);
 int weights_blocks_per_sm();
 
+// group GEMM (gemm.cu)
+int gemm_supported(const Dims &d, int64_t Hp);
+cudaError_t gemm_set_smem_limit();
+int launch_group_gemm(const Dims &d, const moonep_plan_t *plan, const void *x, const void *W, const void *pool,
+                      void *y, int64_t Hp, cudaStream_t st);
+
 // ---- host helpers shared by the entry points (api.cu) ----------------------
 int fail_cuda(cudaError_t e);                  // records the error text, returns MOONEP_ERR_CUDA
 int64_t nvs_of(const moonep_config_t &c);

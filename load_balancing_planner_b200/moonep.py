@@ -59,6 +59,7 @@ def _load():
         "moonep_error_string": ([ctypes.c_int], ctypes.c_char_p),
         "moonep_last_error": ([], ctypes.c_char_p),
         "moonep_plan_noalloc": ([ctypes.POINTER(Config), P, P, ctypes.POINTER(PlanStruct), P], ctypes.c_int),
+        "moonep_group_gemm": ([P, ctypes.POINTER(PlanStruct), P, P, P, P, i64, P], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -70,7 +71,8 @@ def _load():
 lib = _load()
 EXPORTS = ("moonep_create", "moonep_destroy", "moonep_nvs", "moonep_get_config", "moonep_plan",
            "moonep_dispatch", "moonep_combine", "moonep_prefetch_weight", "moonep_reduce_grad",
-           "moonep_read_status", "moonep_error_string", "moonep_last_error", "moonep_plan_noalloc")
+           "moonep_read_status", "moonep_error_string", "moonep_last_error", "moonep_plan_noalloc",
+           "moonep_group_gemm")
 NOALLOC_SCRATCH_BYTES = 1 << 20
 
 
@@ -252,6 +254,22 @@ def moonep_reduce_grad(h: Handle, plan: Plan, grads, reduce_buffers, stream=None
         _expect(RB, (h.R, h.B, h.H, Hp), torch.float32, "reduce_buffers")
     _check(lib.moonep_reduce_grad(h.ptr, ctypes.byref(plan.struct), len(grads), _ptr_array(grads),
                                   _ptr_array(reduce_buffers), Hp, _stream(stream)), "moonep_reduce_grad")
+
+
+def moonep_group_gemm(h: Handle, plan: Plan, x_nvs, weights, pool=None, y_nvs=None, stream=None):
+    """y_nvs [R,NvS,Hp] = x_nvs rows of each plan row @ that row's expert
+    weight (weights [E,H,Hp] bf16 for rows < E, pool [R,B,H,Hp] bf16 for
+    slot rows)."""
+    Hp = weights.shape[-1]
+    _expect(x_nvs, (h.R, h.nvs, h.H), torch.bfloat16, "x_nvs")
+    _expect(weights, (h.E, h.H, Hp), torch.bfloat16, "weights")
+    _expect(pool, (h.R, h.B, h.H, Hp), torch.bfloat16, "pool")
+    if y_nvs is None:
+        y_nvs = torch.empty((h.R, h.nvs, Hp), dtype=torch.bfloat16, device=x_nvs.device)
+    _expect(y_nvs, (h.R, h.nvs, Hp), torch.bfloat16, "y_nvs")
+    _check(lib.moonep_group_gemm(h.ptr, ctypes.byref(plan.struct), _ptr(x_nvs), _ptr(weights), _ptr(pool),
+                                 _ptr(y_nvs), Hp, _stream(stream)), "moonep_group_gemm")
+    return y_nvs
 
 
 def moonep_read_status(plan: Plan, stream=None) -> int:

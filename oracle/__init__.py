@@ -152,3 +152,6 @@ def reduce_grad(slot_expert, G, RB):
     assert G.flags.c_contiguous and RB.flags.c_contiguous
     E, HHp = G.shape
     lib().oracle_reduce_grad(R, B, E, HHp, _p(se), _p(G), _p(RB))
+
+
+from .group_gemm import group_gemm, segments  # noqa: E402,F401  (numpy, fp64)

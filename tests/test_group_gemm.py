@@ -1,0 +1,97 @@
+"""moonep_group_gemm (the VM group GEMM consuming a dispatched layer, MoonEP
+README "Integration", "Weight buffer") against the fp64 oracle on every real
+slot, in training mode (slot rows read the pool) and inference mode (overflow
+rows read the home expert), plus the host-side checks."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from load_balancing_planner_b200 import synth
+from tests.conftest import bf16_to_f64, rel_close
+from tests.gpu_util import bits, gpu_plan, plan_to_numpy, problem
+
+pytestmark = pytest.mark.gpu
+
+
+def _weights(E, H, Hp, seed):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn(E, H, Hp, generator=g) / H ** 0.5).to(torch.bfloat16)
+
+
+def _run(R, S, K, E, B, H, Hp, mode, mv, profile, seed):
+    from load_balancing_planner_b200 import moonep
+    tp = 128
+    tk, tpe, _ = problem(R, S, K, E, mv, profile, seed=seed)
+    h = moonep.moonep_create(S, H, K, E, R, B, tp, mode=mode)
+    p = gpu_plan(h, tk, tpe)
+    x = synth.hidden_bf16(R, S, H, seed=seed).cuda()
+    buf, _ = moonep.moonep_dispatch(h, p, x)
+    W = _weights(E, H, Hp, seed).cuda()
+    pool = torch.zeros((R, max(B, 1), H, Hp), dtype=torch.bfloat16, device="cuda")[:, :B]
+    if B:
+        pool = pool.contiguous()
+        moonep.moonep_prefetch_weight(h, p, [W], [pool])
+    y = moonep.moonep_group_gemm(h, p, buf, W, pool if B else None)
+    torch.cuda.synchronize()
+    assert moonep.moonep_read_status(p) == 0
+    got = plan_to_numpy(p)
+    want, mask = oracle.group_gemm(got["cu_seqlens"], got["row_counts"],
+                                   bits(buf).reshape(R * h.nvs, H), bits(W),
+                                   bits(pool).reshape(R * B, H, Hp) if B else None, E, tp, h.nvs)
+    assert mask.sum() == R * S * K
+    yb = bf16_to_f64(bits(y).reshape(R * h.nvs, Hp)[mask])  # padding slots hold unspecified bits
+    ok = rel_close(yb, want[mask], 1e-2)
+    assert ok.all(), f"{(~ok).sum()} of {ok.size} outside tolerance"
+    h.close()
+    return got
+
+
+@pytest.mark.parametrize("mv", [0.0, 1.0])
+def test_small_training_layer(cuda, mv):
+    got = _run(R=2, S=256, K=4, E=8, B=4, H=128, Hp=256, mode=0, mv=mv, profile="zipf", seed=41)
+    assert (got["slot_expert"] >= 0).any() == (mv > 0)
+
+
+def test_many_k_steps_and_tiles(cuda):
+    # 16 K-steps of 64, 80 row tiles per rank, 2 column tiles, copies from group 0
+    got = _run(R=8, S=1024, K=8, E=64, B=8, H=1024, Hp=512, mode=0, mv=2.0, profile="zipf", seed=42)
+    assert (got["slot_expert"] >= 0).sum() > 4
+
+
+def test_inference_overflow_rows_read_the_home_expert(cuda):
+    got = _run(R=8, S=512, K=8, E=64, B=1, H=256, Hp=256, mode=1, mv=4.0, profile="hot8", seed=43)
+    # some rank holds a remote expert in a home row (overflow past its B slots)
+    G = 64 // 8
+    ovf = [(r, i) for r in range(8) for i in range(64) if got["row_counts"][r, i] and i // G != r]
+    assert ovf
+
+
+def test_failed_plan_and_host_checks(cuda):
+    from load_balancing_planner_b200 import moonep
+    R, S, K, E, B, H, Hp = 2, 128, 2, 8, 4, 128, 256
+    tk, tpe, _ = problem(R, S, K, E, 1.0, "zipf", seed=44)
+    h = moonep.moonep_create(S, H, K, E, R, B, 128)
+    bad = tk.copy()
+    bad[0, 0, 0] = E
+    p = gpu_plan(h, bad)
+    buf = torch.zeros((R, h.nvs, H), dtype=torch.bfloat16, device="cuda")
+    W = _weights(E, H, Hp, 1).cuda()
+    pool = torch.zeros((R, B, H, Hp), dtype=torch.bfloat16, device="cuda")
+    y = torch.full((R, h.nvs, Hp), 7.0, dtype=torch.bfloat16, device="cuda")
+    moonep.moonep_group_gemm(h, p, buf, W, pool, y)
+    torch.cuda.synchronize()
+    assert (y == 7.0).all()  # nothing computed for a failed plan
+    with pytest.raises(ValueError):
+        moonep.moonep_group_gemm(h, p, buf, W[:, :, :128].contiguous(), pool, None)  # pool shape mismatch
+    with pytest.raises(moonep.MoonepError) as e:
+        moonep.moonep_group_gemm(h, p, buf, W[:, :, :128].contiguous(), pool[..., :128].contiguous())
+    assert e.value.code == moonep.ERR_SIZE  # Hp % 256 != 0
+    h.close()
+    h2 = moonep.moonep_create(S, H, K, E, R, B, 64)  # token_padding 64: tiles would straddle rows
+    p2 = gpu_plan(h2, tk, tpe)
+    with pytest.raises(moonep.MoonepError) as e:
+        moonep.moonep_group_gemm(h2, p2, torch.zeros((R, h2.nvs, H), dtype=torch.bfloat16, device="cuda"),
+                                 W, pool)
+    assert e.value.code == moonep.ERR_SIZE
+    h2.close()
