@@ -53,6 +53,10 @@ WORKLOADS = {
     # profiler captures that must stay small
     "train_s512": dict(R=8, S=512, K=8, E=256, B=32, H=7168, tp=128, mode=0, profile="hot8",
                        maxvio=(0.0, 2.0)),
+    # training rows with 64 experts and 1024 tokens per rank: the group GEMM's
+    # profiler case (about 3 GB on the device at H' = 1024)
+    "gemm_small": dict(R=8, S=1024, K=8, E=64, B=8, H=7168, tp=128, mode=0, profile="hot8",
+                       maxvio=(2.0,)),
 }
 
 
@@ -437,7 +441,7 @@ def run_pages_points(w, seed, dev, h, plan, hidden, weights, buf, wn, out, gw, s
     return pts
 
 
-def run_group_gemm_leg(dev, seed, mv=2.0, Hp=2048, reps=10):
+def run_group_gemm_leg(dev, seed, mv=2.0, Hp=2048, reps=10, config="train"):
     """The VM group GEMM that consumes a dispatched training layer: one
     [H, H'] projection per plan row (home experts from W, slot rows from the
     prefetched pool), H' = 2048, bf16 in, fp32 accumulation, bf16 out.
@@ -445,7 +449,7 @@ def run_group_gemm_leg(dev, seed, mv=2.0, Hp=2048, reps=10):
     multiplies each row's padding up to a multiple of 128."""
     import torch
     from load_balancing_planner_b200 import moonep
-    w = WORKLOADS["train"]
+    w = WORKLOADS[config]
     R, S, K, E, B, H, tp = w["R"], w["S"], w["K"], w["E"], w["B"], w["H"], w["tp"]
     tk, real, _ = synth.routing(R, S, K, E, mv, w["profile"], seed=seed)
     h = moonep.moonep_create(S, H, K, E, R, B, tp)
@@ -472,7 +476,7 @@ def run_group_gemm_leg(dev, seed, mv=2.0, Hp=2048, reps=10):
     burst, sustained, kind = tensor_peaks()
     tf = flops / (us * 1e-6) / 1e12
     h.close()
-    return {"workload": f"train shape, plan at maxvio {mv:g}, H'={Hp}, bf16 -> fp32 accumulate -> bf16",
+    return {"workload": f"{config}: {describe(w)}; plan at maxvio {mv:g}, H'={Hp}, bf16 -> fp32 accumulate -> bf16",
             "realised_maxvio": round(real, 4), "flops": flops, "us": round(us, 1), "tflops": round(tf, 1),
             "frac_of_bf16_burst": round(tf / burst, 4), "frac_of_bf16_sustained": round(tf / sustained, 4),
             "peak_kind": kind, "rows_real": R * S * K, "rows_computed": rows_computed}
@@ -739,6 +743,10 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--traffic", type=float, default=None,
                     help="ncu DRAM bytes per launch of the dominant kernel, if measured for this build")
+    ap.add_argument("--gemm-only", action="store_true",
+                    help="time only the group GEMM on the workload (first maxvio of its sweep), for profiler "
+                         "captures; prints the leg's JSON, not a bench line")
+    ap.add_argument("--hp", type=int, default=2048, help="H' of the group GEMM")
     ap.add_argument("--planner-only", action="store_true",
                     help="launch only the planner (every routing of the workload), for profiler captures; "
                          "prints its back-to-back time, not a bench line")
@@ -747,6 +755,12 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.planner_only:
         print(json.dumps(run_planner_only(args)), flush=True)
+        return
+    if args.gemm_only:
+        import torch
+        w = WORKLOADS[args.config]
+        print(json.dumps(run_group_gemm_leg(torch.device("cuda", 0), args.seed, mv=w["maxvio"][0], Hp=args.hp,
+                                            reps=args.steps, config=args.config)), flush=True)
         return
 
     if args.impl == "reference":
