@@ -49,6 +49,9 @@
  *  5. On rank s: row e (e in group s) holds the kept picks of e; the distinct
  *     experts s received, in ascending id, take slots b = 0,1,.. (row E+b);
  *     past B they go to row e itself (inference overflow).  [reading]
+ *     mode 2 (inference, slots by token count): the B received experts with
+ *     the most picks on s take the slots (ties: the lower id), in ascending
+ *     id; the rest overflow.  [reading; the README leaves the choice open]
  *  6. Within a row, picks keep group-sequence order.  Rows are padded to a
  *     multiple of tp (empty rows stay empty); cu_seqlens is the inclusive
  *     running sum of the padded lengths over the E+B rows.  [reading]
@@ -111,7 +114,7 @@ uint16_t oracle_double_to_bf16(double x)
 /*
  * Inputs: topk [R,S,K] int32 (expert ids), tpe [R,E] int32 or NULL (the
  * router's local counts, checked against the picks).  mode 0 = training
- * (B >= E/R), 1 = inference.
+ * (B >= E/R), 1 = inference, 2 = inference with slots by token count.
  * Outputs (caller-allocated): dst [R,S,K], cu_seqlens [R,E+B],
  * row_counts [R,E+B], slot_expert [R,B] (-1 = unused), counts [R,E],
  * maxvio [1], assign [R,4] = {kept, donor group or -1, received start in the
@@ -128,7 +131,7 @@ int oracle_plan(int R, int S, int K, int E, int B, int tp, int mode,
     if (R < 1 || S < 1 || K < 1 || E < 1 || E % R || K > E || B < 0 || tp < 1)
         return ORC_BAD_ARGS;
     const int G = E / R;
-    if (mode == 0 && B < G) return ORC_BAD_ARGS;
+    if (mode < 0 || mode > 2 || (mode == 0 && B < G)) return ORC_BAD_ARGS;
     const int64_t C = (int64_t)S * K;
     const int NR = E + B; /* rows per rank */
     const int64_t NvS = oracle_nvs(S, K, E, R, tp);
@@ -226,6 +229,8 @@ int oracle_plan(int R, int S, int K, int E, int B, int tp, int mode,
         estart[e] = (e % G == 0) ? 0 : estart[e - 1] + T[e - 1];
 
     /* step 5: rows of every rank */
+    int *rx_e = malloc(sizeof(int) * (size_t)G);
+    int64_t *rx_n = malloc(sizeof(int64_t) * (size_t)G);
     memset(row_counts, 0, sizeof(int32_t) * (size_t)R * NR);
     for (int64_t i = 0; i < (int64_t)R * B; i++) slot_expert[i] = -1;
     for (int s = 0; s < R; s++) {
@@ -238,18 +243,34 @@ int oracle_plan(int R, int S, int K, int E, int B, int tp, int mode,
         int h = assign[s * 4 + 1];
         if (h >= 0) {
             int64_t a = assign[s * 4 + 2], b = a + assign[s * 4 + 3];
-            int q = 0;
+            /* the received experts of s in ascending id, with their picks */
+            int nrx = 0;
             for (int e = h * G; e < (h + 1) * G; e++) {
                 int64_t lo = estart[e] > a ? estart[e] : a;
                 int64_t hi = estart[e] + T[e] < b ? estart[e] + T[e] : b;
                 if (hi <= lo) continue;
-                if (q < B) {
-                    slot_expert[(int64_t)s * B + q] = e;
-                    n[E + q] += (int32_t)(hi - lo);
+                rx_e[nrx] = e;
+                rx_n[nrx] = hi - lo;
+                nrx++;
+            }
+            int q = 0;
+            for (int j = 0; j < nrx; j++) {
+                int take;
+                if (mode == 2) { /* rank by picks, more first, ties by lower id */
+                    int better = 0;
+                    for (int m = 0; m < nrx; m++)
+                        if (rx_n[m] > rx_n[j] || (rx_n[m] == rx_n[j] && m < j)) better++;
+                    take = better < B;
                 } else {
-                    n[e] += (int32_t)(hi - lo); /* overflow: the expert's home row */
+                    take = j < B;
                 }
-                q++;
+                if (take) {
+                    slot_expert[(int64_t)s * B + q] = rx_e[j];
+                    n[E + q] += (int32_t)rx_n[j];
+                    q++;
+                } else {
+                    n[rx_e[j]] += (int32_t)rx_n[j]; /* overflow: the expert's home row */
+                }
             }
         }
     }
@@ -292,6 +313,7 @@ int oracle_plan(int R, int S, int K, int E, int B, int tp, int mode,
                     }
     }
 
+    free(rx_n); free(rx_e);
     free(fill); free(estart); free(don_start); free(keep); free(don_amt);
     free(don_to); free(don_from); free(largeq); free(smallq); free(cur);
     free(L); free(T);

@@ -121,7 +121,7 @@ def small_problem(draw):
     K = draw(st.integers(1, min(E, 4)))
     S = draw(st.integers(1, 12))
     tp = draw(st.integers(1, 4))
-    mode = draw(st.integers(0, 1))
+    mode = draw(st.integers(0, 2))
     B = draw(st.integers(G, G + 1)) if mode == 0 else draw(st.integers(0, G))
     seed = draw(st.integers(0, 2 ** 31 - 1))
     hot = draw(st.floats(0.0, 4.0))
@@ -139,6 +139,48 @@ def test_plan_invariants_random(prob):
     p = oracle.plan(tk, E, B, tp, mode)
     assert p["status"] == 0
     check_plan(tk, p, E, B, tp, mode)
+    if mode:
+        _check_slot_choice(p, E, B, tk.shape[0], by_count=mode == 2)
+
+
+def _check_slot_choice(p, E, B, R, by_count):
+    """Inference slots: in ascending id; by id (mode 1) they hold the lowest
+    ids among the received experts, by count (mode 2) no overflow expert has
+    more picks on the rank than a slot expert, and on a tie the slot expert
+    has the lower id."""
+    G = E // R
+    rc, se = p["row_counts"], p["slot_expert"]
+    for r in range(R):
+        slots = [int(e) for e in se[r] if e >= 0]
+        assert slots == sorted(slots)
+        got = {e: int(rc[r, E + b]) for b, e in enumerate(slots)}
+        ovf = {e: int(rc[r, e]) for e in range(E) if e // G != r and rc[r, e] > 0}
+        for e, n in got.items():
+            for f, m in ovf.items():
+                if by_count:
+                    assert n > m or (n == m and e < f), (r, e, n, f, m)
+                else:
+                    assert e < f
+
+
+def test_inference_slots_by_count_and_by_id():
+    # training-shape inference at maxvio 4: ranks receive more distinct
+    # experts than B = 4, so the two rules must pick differently somewhere
+    tk, mv, _ = synth.routing(8, 4096, 8, 256, 4.0, "hot8", 0)
+    p1 = oracle.plan(tk, 256, 4, 128, 1)
+    p2 = oracle.plan(tk, 256, 4, 128, 2)
+    for p, by_count in ((p1, False), (p2, True)):
+        assert p["status"] == 0
+        check_plan(tk, p, 256, 4, 128, 1)
+        _check_slot_choice(p, 256, 4, 8, by_count)
+    assert not np.array_equal(p1["slot_expert"], p2["slot_expert"])
+    # the per-expert totals and the alias chain do not depend on the rule
+    assert np.array_equal(p1["assign"], p2["assign"]) and np.array_equal(p1["counts"], p2["counts"])
+    # with enough slots for every received expert the two rules coincide
+    q1 = oracle.plan(tk, 256, 32, 128, 1)
+    q2 = oracle.plan(tk, 256, 32, 128, 2)
+    for k in ("dst", "cu_seqlens", "row_counts", "slot_expert"):
+        assert np.array_equal(q1[k], q2[k]), k
 
 
 # ------------------------------------------------ special cases: stable sort

@@ -37,7 +37,7 @@ MUTANTS = {
     "maxvio sign": ("*maxvio = (float)((double)maxT / Tbar - 1.0);",
                     "*maxvio = (float)((double)maxT / Tbar + 1.0);"),
     "slots in descending order": (
-        "slot_expert[(int64_t)s * B + q] = e;", "slot_expert[(int64_t)s * B + (B - 1 - q)] = e;"),
+        "slot_expert[(int64_t)s * B + q] = rx_e[j];", "slot_expert[(int64_t)s * B + (B - 1 - q)] = rx_e[j];"),
     "consumed slots not zeroed": (
         "for (int64_t i = 0; i < HHp; i++) RB[holders[j] * HHp + i] = 0.0f;", "(void)0;"),
     "reduction adds one slot": (
@@ -52,8 +52,14 @@ MUTANTS = {
         "                    for (int k = 0; k < K; k++) {\n                        int64_t idx"),
     "duplicate check off": ("if (tok[k2] == e) status |= ORC_DUP_EXPERT;", "(void)0;"),
     "overflow goes to the last slot": (
-        "n[e] += (int32_t)(hi - lo); /* overflow: the expert's home row */",
-        "n[E + B - 1] += (int32_t)(hi - lo);"),
+        "n[rx_e[j]] += (int32_t)rx_n[j]; /* overflow: the expert's home row */",
+        "n[E + B - 1] += (int32_t)rx_n[j];"),
+    "slots by count take the fewest picks": (
+        "if (rx_n[m] > rx_n[j] || (rx_n[m] == rx_n[j] && m < j)) better++;",
+        "if (rx_n[m] < rx_n[j] || (rx_n[m] == rx_n[j] && m < j)) better++;"),
+    "slots by count break ties to the higher id": (
+        "if (rx_n[m] > rx_n[j] || (rx_n[m] == rx_n[j] && m < j)) better++;",
+        "if (rx_n[m] > rx_n[j] || (rx_n[m] == rx_n[j] && m > j)) better++;"),
 }
 
 
