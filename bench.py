@@ -519,9 +519,20 @@ def run_legs(args, dev, world):
         D = int(np.unique(se[se >= 0]).size)
         ms = timed(lambda: moonep.moonep_prefetch_weight(h, p, Ws, pools))
         by = 3 * (D + U) * H * Hp * 2
+        # picks left on overflow rows (weights read from the home rank), with
+        # the slots given by id (mode 1, timed here) and by picks (mode 2)
+        ovf = {}
+        for mode in (1, 2):
+            hm = moonep.moonep_create(S, H, K, E, R, 4, tp, mode=mode)
+            pm = moonep.moonep_plan(hm, torch.from_numpy(tk).to(dev),
+                                    torch.from_numpy(synth.local_counts(tk, E)).to(dev))
+            rc = pm.row_counts.cpu().numpy()
+            ovf[mode] = int(sum(rc[r, e] for r in range(R) for e in range(E) if e // (E // R) != r))
+            hm.close()
         out[f"{mv:g}"] = dict(realised_maxvio=round(real, 4), used_slots=U, distinct_experts=D,
                               us=round(ms * 1e3, 1), gbs=round(by / (ms * 1e-3) / 1e9, 1),
-                              frac_measured=round(by / (ms * 1e-3) / 1e9 / peak, 4))
+                              frac_measured=round(by / (ms * 1e-3) / 1e9 / peak, 4),
+                              overflow_picks_slots_by_id=ovf[1], overflow_picks_slots_by_count=ovf[2])
     legs["prefetch_weight"] = dict(workload="inference R=8 S=4096 K=8 E=256 B=4 H=7168 H'=2048, 3 projections",
                                    bytes="3*(D+U)*H*H'*2", points=out)
     del Ws, pools

@@ -78,7 +78,12 @@ typedef struct CUstream_st *moonep_stream_t;
  *   mode             : 0 = training, which needs B >= E/R because copies come
  *                      from at most one remote home group per rank; 1 =
  *                      inference, any B >= 0, copied experts past the first B
- *                      are read from their home rows ("How to set B").
+ *                      are read from their home rows ("How to set B"); 2 =
+ *                      inference where the B slots go to the received experts
+ *                      with the most picks on the rank (ties: lower id), so
+ *                      the home-row overflow carries the fewest tokens (the
+ *                      README leaves this choice open).  Slots are in
+ *                      ascending expert id in every mode.
  */
 typedef struct {
     int32_t S, H, K, E, R, B, token_padding, num_sms, mode;

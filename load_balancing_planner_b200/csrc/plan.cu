@@ -595,35 +595,57 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
             }
             carry = __shfl_sync(0xffffffffu, incl, 31);
         }
-        int nq = 0, ocarry = 0, scarry = 0;
+        int nq = 0, nslot = 0, ocarry = 0, scarry = 0;
         const int h = s_rfrom[s];
         if (h >= 0) {
             const int a0 = s_rstart[s], a1 = a0 + s_rlen[s];
+            // Which received experts take the B slots: the first B in id
+            // order, or (mode 2) the B with the most picks here, ties to the
+            // lower id; the slots themselves go in id order either way.
+            const bool by_count = d.mode == 2;
+            if (by_count) {
+                for (int j = lane; j < G; j += 32) {
+                    const int e = h * G + j;
+                    nrecv[s * G + j] = max(0, min(es[e] + T[e], a1) - max(es[e], a0));
+                }
+                __syncwarp();
+            }
             for (int j0 = 0; j0 < G; j0 += 32) {
                 const int j = j0 + lane;
                 const int e = h * G + j;
                 int ov = 0;
                 if (j < G) ov = max(0, min(es[e] + T[e], a1) - max(es[e], a0));
                 const unsigned has = __ballot_sync(0xffffffffu, ov > 0);
-                const int q = nq + __popc(has & lanemask_lt());
-                const bool is_slot = ov > 0 && q < B, is_ovf = ov > 0 && q >= B;
+                bool take = ov > 0 && nq + __popc(has & lanemask_lt()) < B;
+                if (by_count && ov > 0) {
+                    int better = 0;
+                    for (int m = 0; m < G; ++m) {
+                        const int om = nrecv[s * G + m];
+                        better += (om > ov) || (om == ov && m < j);
+                    }
+                    take = better < B;
+                }
+                const unsigned tk = __ballot_sync(0xffffffffu, take);
+                // slot index of a taken expert; B marks an overflow row
+                const int q = take ? nslot + __popc(tk & lanemask_lt()) : B;
+                const bool is_ovf = ov > 0 && !take;
                 const int oincl = warp_incl_scan(is_ovf ? pad_to(ov, tp) : 0) + ocarry;
-                const int sincl = warp_incl_scan(is_slot ? pad_to(ov, tp) : 0) + scarry;
+                const int sincl = warp_incl_scan(take ? pad_to(ov, tp) : 0) + scarry;
                 if (j < G) {
                     nrecv[s * G + j] = ov;
                     qidx[s * G + j] = (int16_t)(ov > 0 ? q : -1);
                     ovfincl[s * G + j] = oincl;
                 }
-                if (is_slot) {
+                if (take) {
                     slotj[s * B + q] = (int16_t)j;
                     slotincl[s * B + q] = sincl;
                 }
                 nq += __popc(has);
+                nslot += __popc(tk);
                 ocarry = __shfl_sync(0xffffffffu, oincl, 31);
                 scarry = __shfl_sync(0xffffffffu, sincl, 31);
             }
         }
-        const int nslot = min(nq, B);
         for (int b = nslot + lane; b < B; b += 32) {
             slotj[s * B + b] = (int16_t)-1;
             slotincl[s * B + b] = scarry;

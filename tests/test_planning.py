@@ -19,6 +19,9 @@ CASES = [
     # donated picks span two recipients
     ("train_skew", 8, 4096, 8, 256, 32, 128, 0, "hot8", [10.0, 20.0]),
     ("infer", 8, 4096, 8, 256, 4, 128, 1, "hot8", [1.0, 4.0, 20.0]),
+    # inference with the slots given to the most-picked received experts
+    ("infer_count", 8, 4096, 8, 256, 4, 128, 2, "hot8", [1.0, 4.0, 20.0]),
+    ("infer_count_wide", 4, 600, 8, 1024, 2, 64, 2, "hot8", [4.0]),
     ("ragged", 3, 1000, 3, 24, 8, 16, 0, "hot8", [1.5]),
     ("one_rank", 1, 700, 4, 16, 16, 8, 0, "zipf", [2.0]),
     ("k1_tp1", 8, 64, 1, 8, 1, 1, 0, "boost0", [3.0]),
@@ -112,7 +115,7 @@ def test_random_small_plans_match_oracle(cuda):
         K = int(g.integers(1, min(E, 4) + 1))
         S = int(g.integers(1, 41))
         tp = int(g.integers(1, 5))
-        mode = int(g.integers(0, 2))
+        mode = int(g.integers(0, 3))
         B = int(g.integers(G, G + 2)) if mode == 0 else int(g.integers(0, G + 1))
         w = np.ones(E)
         w[g.integers(0, E)] += g.uniform(0, 4) * E
@@ -124,3 +127,18 @@ def test_random_small_plans_match_oracle(cuda):
         got = plan_to_numpy(gpu_plan(h, tk))
         assert_plans_equal(got, want)
         h.close()
+
+
+def test_inference_slot_rules_differ_on_gpu_as_in_the_oracle(cuda):
+    # mode 1 (slots by id) and mode 2 (slots by picks) on the same routing:
+    # each GPU plan equals its oracle plan, and the two rules choose differently
+    from load_balancing_planner_b200 import moonep
+    R, S, K, E, B, tp = 8, 4096, 8, 256, 4, 128
+    tk, tpe, _ = problem(R, S, K, E, 20.0, "hot8", seed=11)
+    got = {}
+    for mode in (1, 2):
+        h = moonep.moonep_create(S, 8, K, E, R, B, tp, mode=mode)
+        got[mode] = plan_to_numpy(gpu_plan(h, tk, tpe))
+        assert_plans_equal(got[mode], oracle.plan(tk, E, B, tp, mode, tpe))
+        h.close()
+    assert not np.array_equal(got[1]["slot_expert"], got[2]["slot_expert"])
