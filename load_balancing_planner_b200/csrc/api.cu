@@ -277,7 +277,7 @@ extern "C" int moonep_prefetch_weight(moonep_handle_t h, const moonep_plan_t *pl
     const int rc = weight_args(h, plan, n_proj, weights, pool, Hp, &a);
     if (rc != MOONEP_OK) return rc;
     if (h->d.B == 0) return MOONEP_OK;  // no slots: nothing to copy
-    const cudaError_t e = launch_prefetch(a, h->grid_weights, reinterpret_cast<cudaStream_t>(stream));
+    const cudaError_t e = launch_prefetch(a, h->grid_weights, h->sms, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? MOONEP_OK : fail_cuda(e);
 }
 

@@ -147,6 +147,78 @@ __global__ void __launch_bounds__(kWThreads) prefetch_kernel(WeightArgs a) {
     }
 }
 
+// Bulk variant of the prefetch: after the block has built the slot lists,
+// one thread moves 32 KB pieces of each expert matrix through a 3-stage ring
+// in shared memory with the TMA engine: one bulk load per piece, then one
+// bulk store per slot holding the expert, and the stage is refilled as soon
+// as those stores have read it.  Every expert piece is read once.
+constexpr int kPfStages = 3;
+constexpr uint32_t kPfTile = 32 * 1024;
+
+__global__ void __launch_bounds__(kWThreads) prefetch_bulk_kernel(WeightArgs a) {
+    pdl_wait();
+    if (*a.status != 0) return;
+    extern __shared__ __align__(128) int32_t wsm[];
+    const int RB = a.d.R * a.d.B;
+    int32_t *se = wsm, *nxt = wsm + RB, *lead = wsm + 2 * RB;
+    const int nlead = build_slot_lists(a, se, nxt, lead);
+    if (nlead <= 0 || threadIdx.x != 0) return;
+    uint8_t *stages = reinterpret_cast<uint8_t *>(wsm) + ((sizeof(int32_t) * 3 * (size_t)RB + 127) & ~(size_t)127);
+    const uint32_t stage0 = smem_addr(stages);
+    const uint32_t bar0 = stage0 + kPfStages * kPfTile;
+    const uint64_t bytes_per = (uint64_t)a.hhp * 2;  // one expert matrix, bf16
+    const int64_t ntiles = (int64_t)((bytes_per + kPfTile - 1) / kPfTile);
+    const int64_t units = (int64_t)a.n_proj * nlead * ntiles;
+    const int64_t first = blockIdx.x, step = gridDim.x;
+    const uint64_t pol = l2_evict_first_policy();
+    // unit i of this block -> projection, leading slot, byte offset, size
+    auto piece = [&](int64_t i, int &p, int &s, uint64_t &off, uint32_t &n) {
+        const int64_t u = first + i * step;
+        p = (int)(u / ((int64_t)nlead * ntiles));
+        const int64_t rem = u - (int64_t)p * nlead * ntiles;
+        s = lead[rem / ntiles];
+        off = (uint64_t)(rem % ntiles) * kPfTile;
+        n = (uint32_t)min((uint64_t)kPfTile, bytes_per - off);
+    };
+    auto load = [&](int64_t i, int st) {
+        int p, s;
+        uint64_t off;
+        uint32_t n;
+        piece(i, p, s, off, n);
+        bulk_load(stage0 + st * kPfTile, static_cast<const uint8_t *>(a.src[p]) + (uint64_t)se[s] * bytes_per + off,
+                  n, bar0 + 8u * st);
+    };
+    for (int st = 0; st < kPfStages; ++st) mbar_init(bar0 + 8u * st);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    for (int st = 0; st < kPfStages; ++st)
+        if (first + st * step < units) load(st, st);
+    bool ok = true;
+    int64_t i = 0;
+    for (; first + i * step < units; ++i) {
+        const int st = (int)(i % kPfStages);
+        if (!(ok = mbar_wait(bar0 + 8u * st, (uint32_t)((i / kPfStages) & 1)))) break;
+        int p, s;
+        uint64_t off;
+        uint32_t n;
+        piece(i, p, s, off, n);
+        for (int j = s; j >= 0; j = nxt[j])
+            bulk_store(static_cast<uint8_t *>(a.dst[p]) + (uint64_t)j * bytes_per + off, stage0 + st * kPfTile, n, pol);
+        bulk_commit();
+        // refill the previous unit's stage once its stores have read it
+        if (i >= 1 && first + (i - 1 + kPfStages) * step < units) {
+            bulk_wait_read1();
+            load(i - 1 + kPfStages, (int)((i - 1) % kPfStages));
+        }
+    }
+    if (!ok) {
+        atomicOr(a.status, MOONEP_STATUS_TIMEOUT);
+        // loads still in flight: units i .. i + kPfStages - 2 (bounded waits)
+        for (int64_t j = i; j < i + kPfStages - 1 && first + j * step < units; ++j)
+            mbar_wait(bar0 + 8u * (uint32_t)(j % kPfStages), (uint32_t)((j / kPfStages) & 1));
+    }
+    bulk_wait_all();
+}
+
 // a.src[p] = reduce buffer [R*B, H*Hp] (read, then zeroed), a.dst[p] = grads [E, H*Hp].
 __global__ void __launch_bounds__(kWThreads) reduce_grad_kernel(WeightArgs a) {
     pdl_wait();
@@ -220,8 +292,33 @@ static cudaError_t launch_w(Kern kern, const WeightArgs &a, int grid, cudaStream
     return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
-cudaError_t launch_prefetch(const WeightArgs &a, int grid, cudaStream_t st) {
-    return launch_w(prefetch_kernel, a, grid, st);
+static size_t prefetch_bulk_smem(const WeightArgs &a) {
+    return ((weights_smem(a) + 127) & ~(size_t)127) + kPfStages * (size_t)kPfTile + 8 * kPfStages;
+}
+
+// The bulk prefetch needs 16-byte aligned matrices of whole 16-byte units and
+// room for its ring next to the slot tables.
+bool prefetch_use_bulk(const WeightArgs &a) {
+    bool aligned = ((a.hhp * 2) % 16) == 0;
+    for (int p = 0; p < a.n_proj; ++p)
+        aligned = aligned && (reinterpret_cast<uintptr_t>(a.src[p]) % 16) == 0 &&
+                  (reinterpret_cast<uintptr_t>(a.dst[p]) % 16) == 0;
+    return aligned && a.hhp * 2 >= kPfTile && prefetch_bulk_smem(a) <= 110 * 1024;
+}
+
+cudaError_t launch_prefetch(const WeightArgs &a, int grid, int sms, cudaStream_t st) {
+    if (!prefetch_use_bulk(a)) return launch_w(prefetch_kernel, a, grid, st);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(2 * sms));  // two rings per SM
+    cfg.blockDim = dim3(kWThreads);
+    cfg.dynamicSmemBytes = prefetch_bulk_smem(a);
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, prefetch_bulk_kernel, a);
 }
 
 cudaError_t launch_reduce_grad(const WeightArgs &a, int grid, cudaStream_t st) {
@@ -244,6 +341,8 @@ size_t weights_static_smem_bytes() {
 
 cudaError_t weights_set_smem_limit(size_t bytes) {
     cudaError_t e = cudaFuncSetAttribute(prefetch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(prefetch_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e != cudaSuccess) return e;
     return cudaFuncSetAttribute(reduce_grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }

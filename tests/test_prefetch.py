@@ -66,3 +66,26 @@ def test_prefetch_inference_shape_full(cuda):
     rc = o["row_counts"]
     assert any(rc[r, e] > 0 for r in range(R) for e in range(E) if e // 32 != r)
     h.close()
+
+
+@pytest.mark.parametrize("H,Hp", [(136, 200), (256, 128)])
+def test_prefetch_bulk_path_with_a_ragged_last_piece(cuda, H, Hp):
+    # expert matrices of 54,400 and 65,536 bytes: moved in 32 KB bulk pieces,
+    # the first with a shorter last piece
+    from load_balancing_planner_b200 import moonep
+    R, S, K, E, B, tp = 8, 1024, 8, 64, 8, 128
+    tk, tpe, _ = problem(R, S, K, E, 2.0, "hot8", seed=5)
+    h = moonep.moonep_create(S, H, K, E, R, B, tp)
+    p = gpu_plan(h, tk, tpe)
+    Ws = [synth.hidden_bf16(1, E, H * Hp, seed=30 + i).view(E, H, Hp) for i in range(2)]
+    pools = [torch.empty((R, B, H, Hp), dtype=torch.int16, device="cuda").fill_(0x7F7F).view(torch.bfloat16)
+             for _ in range(2)]
+    moonep.moonep_prefetch_weight(h, p, [W.cuda() for W in Ws], pools)
+    torch.cuda.synchronize()
+    assert moonep.moonep_read_status(p) == 0
+    o = oracle.plan(tk, E, B, tp, 0, tpe)
+    for W, pool in zip(Ws, pools):
+        opool = np.full((R * B, H * Hp), 0x7F7F, np.uint16)
+        oracle.prefetch(o["slot_expert"], synth.bf16_bits(W).reshape(E, H * Hp), opool)
+        assert np.array_equal(bits(pool).reshape(R * B, H * Hp), opool)
+    h.close()
