@@ -290,7 +290,7 @@ extern "C" int moonep_reduce_grad(moonep_handle_t h, const moonep_plan_t *plan, 
                                reinterpret_cast<void *const *>(grads), Hp, &a);
     if (rc != MOONEP_OK) return rc;
     if (h->d.B == 0) return MOONEP_OK;
-    const cudaError_t e = launch_reduce_grad(a, h->grid_weights, reinterpret_cast<cudaStream_t>(stream));
+    const cudaError_t e = launch_reduce_grad(a, h->grid_weights, h->sms, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? MOONEP_OK : fail_cuda(e);
 }
 

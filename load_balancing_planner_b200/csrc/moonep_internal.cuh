@@ -84,7 +84,7 @@ struct WeightArgs {
 };
 
 cudaError_t launch_prefetch(const WeightArgs &a, int grid, int sms, cudaStream_t st);
-cudaError_t launch_reduce_grad(const WeightArgs &a, int grid, cudaStream_t st);
+cudaError_t launch_reduce_grad(const WeightArgs &a, int grid, int sms, cudaStream_t st);
 int weights_blocks_per_sm();
 
 // group GEMM (gemm.cu)

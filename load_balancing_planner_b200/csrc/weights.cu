@@ -17,6 +17,7 @@ namespace moonep {
 constexpr int kWThreads = 256;
 constexpr int kWVec = 4;                          // 16-byte vectors per thread per tile
 constexpr int kWTile = kWThreads * kWVec;         // vectors per tile
+constexpr int kWMaxWarps = 9;                     // warps of the largest block that builds slot lists
 
 // Binary search for expert e in one rank's slot row: used slots first, in
 // ascending expert order, then -1s (the layout moonep_plan writes).
@@ -44,20 +45,21 @@ __device__ __forceinline__ int warp_incl_scan_w(int v) {
 // Shared-memory slot tables: se[RB] expert or -1, nxt[RB] next slot holding
 // the same expert (-1 = last), lead[] leading slots in ascending order.
 // Returns the number of leaders, or -1 after flagging a malformed slot table.
-__device__ int build_slot_lists(const WeightArgs &a, int32_t *se, int32_t *nxt, int32_t *lead) {
+__device__ int build_slot_lists(const WeightArgs &a, int32_t *se, int32_t *nxt, int32_t *lead,
+                                int nthreads = kWThreads) {
     __shared__ int s_bad;
-    __shared__ int s_warp[kWThreads / 32];
+    __shared__ int s_warp[kWMaxWarps];
     const int R = a.d.R, B = a.d.B, E = a.d.E, RB = R * B;
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     if (tid == 0) s_bad = 0;
     __syncthreads();
-    for (int s = tid; s < RB; s += kWThreads) {
+    for (int s = tid; s < RB; s += nthreads) {
         const int e = a.slot_expert[s];
         if (e < -1 || e >= E) s_bad = 1;
         se[s] = e;
     }
     __syncthreads();
-    for (int s = tid; s < RB; s += kWThreads) {
+    for (int s = tid; s < RB; s += nthreads) {
         const int e = se[s];
         if (s % B != 0 && e >= 0) {
             const int prev = se[s - 1];
@@ -69,7 +71,7 @@ __device__ int build_slot_lists(const WeightArgs &a, int32_t *se, int32_t *nxt, 
         if (tid == 0) atomicOr(a.status, MOONEP_STATUS_BAD_PLAN);
         return -1;
     }
-    const int per = (RB + kWThreads - 1) / kWThreads;  // <= 16 (RB <= 4096)
+    const int per = (RB + nthreads - 1) / nthreads;  // <= 32 (RB <= 8192)
     const int s0 = min(RB, tid * per), s1 = min(RB, s0 + per);
     unsigned mask = 0;
     int cnt = 0;
@@ -99,14 +101,15 @@ __device__ int build_slot_lists(const WeightArgs &a, int32_t *se, int32_t *nxt, 
     const int incl = warp_incl_scan_w(cnt);
     if (lane == 31) s_warp[w] = incl;
     __syncthreads();
+    const int nw = nthreads / 32;
     if (w == 0) {
-        const int x = lane < kWThreads / 32 ? s_warp[lane] : 0;
+        const int x = lane < nw ? s_warp[lane] : 0;
         const int xi = warp_incl_scan_w(x);
-        if (lane < kWThreads / 32) s_warp[lane] = xi;
+        if (lane < nw) s_warp[lane] = xi;
     }
     __syncthreads();
     int pos = (w > 0 ? s_warp[w - 1] : 0) + incl - cnt;
-    const int total = s_warp[kWThreads / 32 - 1];
+    const int total = s_warp[nw - 1];
     for (int s = s0; s < s1; ++s)
         if (mask & (1u << (s - s0))) lead[pos++] = s;
     __syncthreads();
@@ -275,6 +278,138 @@ __global__ void __launch_bounds__(kWThreads) reduce_grad_kernel(WeightArgs a) {
     }
 }
 
+// Bulk variant of the grad-slot reduction.  Warp 0 streams, one 16 KB fp32
+// piece at a time, each unit's grad piece and then its holders' pieces in
+// ascending slot order through a 6-slot ring in shared memory (bulk loads
+// completing on mbarriers); the other 8 warps add them up in registers (16
+// floats a thread), in that order, store the sum to the grad and zeros to
+// the holders, and hand each ring slot back as soon as they have read it.
+constexpr int kRgRing = 6;
+constexpr int kRgTile = 4096;                  // floats per piece (16 KB)
+constexpr int kRgThreads = 32 + 256;           // producer warp + 8 summing warps
+constexpr int kRgPer = kRgTile / 256;          // floats per summing thread
+
+__global__ void __launch_bounds__(kRgThreads) reduce_grad_bulk_kernel(WeightArgs a) {
+    pdl_wait();
+    if (*a.status != 0) return;
+    extern __shared__ __align__(128) int32_t wsm[];
+    const int RB = a.d.R * a.d.B;
+    int32_t *se = wsm, *nxt = wsm + RB, *lead = wsm + 2 * RB;
+    const int nlead = build_slot_lists(a, se, nxt, lead, kRgThreads);
+    if (nlead <= 0) return;
+    uint8_t *ring = reinterpret_cast<uint8_t *>(wsm) + ((sizeof(int32_t) * 3 * (size_t)RB + 127) & ~(size_t)127);
+    const uint32_t ring0 = smem_addr(ring);
+    const uint32_t full0 = ring0 + kRgRing * kRgTile * 4, empty0 = full0 + 8 * kRgRing;
+    const int64_t npiece = (a.hhp + kRgTile - 1) / kRgTile;
+    const int64_t units = (int64_t)a.n_proj * nlead * npiece;
+    const int64_t first = blockIdx.x, step = gridDim.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    __shared__ int s_err;
+    if (tid == 0) {
+        s_err = 0;
+        for (int k = 0; k < kRgRing; ++k) {
+            mbar_init(full0 + 8u * k);
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(empty0 + 8u * k), "r"(8) : "memory");
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    volatile int *err = &s_err;
+    auto unit = [&](int64_t i, int &p, int &s, int64_t &off, int &n) {
+        const int64_t u = first + i * step;
+        p = (int)(u / ((int64_t)nlead * npiece));
+        const int64_t rem = u - (int64_t)p * nlead * npiece;
+        s = lead[rem / npiece];
+        off = (rem % npiece) * kRgTile;
+        n = (int)min((int64_t)kRgTile, a.hhp - off);
+    };
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int64_t seq = 0;  // pieces issued: ring slot seq % kRgRing, round seq / kRgRing
+            for (int64_t i = 0; first + i * step < units && !*err; ++i) {
+                int p, s, n;
+                int64_t off;
+                unit(i, p, s, off, n);
+                const float *g = static_cast<const float *>(a.dst[p]) + (int64_t)se[s] * a.hhp + off;
+                const float *rb = static_cast<const float *>(a.src[p]) + off;
+                // the unit's pieces: its grad (j = -1), then every holder in slot order
+                for (int j = -1;;) {
+                    const int k = (int)(seq % kRgRing);
+                    if (seq >= kRgRing && !mbar_wait(empty0 + 8u * k, (uint32_t)(((seq / kRgRing) - 1) & 1))) {
+                        atomicOr(a.status, MOONEP_STATUS_TIMEOUT);
+                        *err = 1;
+                        break;
+                    }
+                    bulk_load(ring0 + k * kRgTile * 4, j < 0 ? g : rb + (int64_t)j * a.hhp, (uint32_t)n * 4u,
+                              full0 + 8u * k);
+                    ++seq;
+                    j = j < 0 ? s : nxt[j];
+                    if (j < 0) break;
+                }
+            }
+            // the last load issued into each ring slot has landed before anyone leaves
+            for (int64_t q = max((int64_t)0, seq - kRgRing); q < seq; ++q)
+                if (!mbar_wait(full0 + 8u * (uint32_t)(q % kRgRing), (uint32_t)((q / kRgRing) & 1)))
+                    atomicOr(a.status, MOONEP_STATUS_TIMEOUT);
+        }
+        return;
+    }
+    const int t = tid - 32;  // summing thread 0..255
+    int64_t seq = 0;
+    for (int64_t i = 0; first + i * step < units && !*err; ++i) {
+        int p, s, n;
+        int64_t off;
+        unit(i, p, s, off, n);
+        float acc[kRgPer];
+        bool ok = true;
+        for (int j = -1;;) {  // the grad piece, then every holder in slot order
+            const int k = (int)(seq % kRgRing);
+            ok = __all_sync(0xffffffffu, mbar_wait(full0 + 8u * k, (uint32_t)((seq / kRgRing) & 1)));
+            if (!ok) break;
+            const float4 *v = reinterpret_cast<const float4 *>(ring + (size_t)k * kRgTile * 4);
+#pragma unroll
+            for (int q = 0; q < kRgPer / 4; ++q) {
+                const int idx = q * 256 + t;  // float4 index inside the piece
+                const float4 x = idx * 4 < n ? v[idx] : make_float4(0.f, 0.f, 0.f, 0.f);
+                if (j < 0) {
+                    acc[4 * q] = x.x, acc[4 * q + 1] = x.y, acc[4 * q + 2] = x.z, acc[4 * q + 3] = x.w;
+                } else {
+                    acc[4 * q] = __fadd_rn(acc[4 * q], x.x);
+                    acc[4 * q + 1] = __fadd_rn(acc[4 * q + 1], x.y);
+                    acc[4 * q + 2] = __fadd_rn(acc[4 * q + 2], x.z);
+                    acc[4 * q + 3] = __fadd_rn(acc[4 * q + 3], x.w);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(empty0 + 8u * k) : "memory");
+            ++seq;
+            j = j < 0 ? s : nxt[j];
+            if (j < 0) break;
+        }
+        if (!ok) {
+            if (lane == 0) atomicOr(a.status, MOONEP_STATUS_TIMEOUT);
+            *err = 1;
+            break;
+        }
+        float4 *g = reinterpret_cast<float4 *>(static_cast<float *>(a.dst[p]) + (int64_t)se[s] * a.hhp + off);
+#pragma unroll
+        for (int q = 0; q < kRgPer / 4; ++q) {
+            const int idx = q * 256 + t;
+            if (idx * 4 < n) __stcs(g + idx, make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]));
+        }
+        const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = s; j >= 0; j = nxt[j]) {
+            float4 *z = reinterpret_cast<float4 *>(static_cast<float *>(const_cast<void *>(a.src[p])) + (int64_t)j * a.hhp + off);
+#pragma unroll
+            for (int q = 0; q < kRgPer / 4; ++q) {
+                const int idx = q * 256 + t;
+                if (idx * 4 < n) __stcs(z + idx, zero);
+            }
+        }
+    }
+}
+
 static size_t weights_smem(const WeightArgs &a) { return sizeof(int32_t) * 3 * (size_t)a.d.R * a.d.B; }
 
 template <typename Kern>
@@ -321,8 +456,31 @@ cudaError_t launch_prefetch(const WeightArgs &a, int grid, int sms, cudaStream_t
     return cudaLaunchKernelEx(&cfg, prefetch_bulk_kernel, a);
 }
 
-cudaError_t launch_reduce_grad(const WeightArgs &a, int grid, cudaStream_t st) {
-    return launch_w(reduce_grad_kernel, a, grid, st);
+static size_t reduce_bulk_smem(const WeightArgs &a) {
+    return ((weights_smem(a) + 127) & ~(size_t)127) + kRgRing * (size_t)kRgTile * 4 + 16 * kRgRing;
+}
+
+bool reduce_grad_use_bulk(const WeightArgs &a) {
+    bool aligned = (a.hhp % 4) == 0;
+    for (int p = 0; p < a.n_proj; ++p)
+        aligned = aligned && (reinterpret_cast<uintptr_t>(a.src[p]) % 16) == 0 &&
+                  (reinterpret_cast<uintptr_t>(a.dst[p]) % 16) == 0;
+    return aligned && a.hhp >= kRgTile && reduce_bulk_smem(a) <= 110 * 1024;
+}
+
+cudaError_t launch_reduce_grad(const WeightArgs &a, int grid, int sms, cudaStream_t st) {
+    if (!reduce_grad_use_bulk(a)) return launch_w(reduce_grad_kernel, a, grid, st);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(2 * sms));  // two rings per SM
+    cfg.blockDim = dim3(kRgThreads);
+    cfg.dynamicSmemBytes = reduce_bulk_smem(a);
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, reduce_grad_bulk_kernel, a);
 }
 
 int weights_blocks_per_sm() {
@@ -336,6 +494,9 @@ size_t weights_static_smem_bytes() {
     size_t m = 0;
     if (cudaFuncGetAttributes(&fa, prefetch_kernel) == cudaSuccess) m = fa.sharedSizeBytes;
     if (cudaFuncGetAttributes(&fa, reduce_grad_kernel) == cudaSuccess && fa.sharedSizeBytes > m) m = fa.sharedSizeBytes;
+    if (cudaFuncGetAttributes(&fa, prefetch_bulk_kernel) == cudaSuccess && fa.sharedSizeBytes > m) m = fa.sharedSizeBytes;
+    if (cudaFuncGetAttributes(&fa, reduce_grad_bulk_kernel) == cudaSuccess && fa.sharedSizeBytes > m)
+        m = fa.sharedSizeBytes;
     return m;
 }
 
@@ -343,6 +504,8 @@ cudaError_t weights_set_smem_limit(size_t bytes) {
     cudaError_t e = cudaFuncSetAttribute(prefetch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(prefetch_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(reduce_grad_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e != cudaSuccess) return e;
     return cudaFuncSetAttribute(reduce_grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }

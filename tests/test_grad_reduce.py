@@ -20,6 +20,9 @@ RTOL_F32 = 1e-5
     (8, 1024, 8, 64, 8, 128, 0, 2.0, 64, 64, 1),
     (8, 1024, 8, 64, 3, 128, 1, 2.0, 8, 36, 3),
     (3, 1000, 3, 24, 8, 16, 0, 1.5, 24, 20, 1),
+    # 16 KB pieces through the bulk path, the last one short
+    (8, 1024, 8, 64, 8, 128, 0, 2.0, 72, 100, 2),
+    (8, 1024, 8, 64, 3, 128, 1, 4.0, 128, 64, 3),
 ])
 def test_reduce_grad_matches_oracle(cuda, R, S, K, E, B, tp, mode, mv, H, Hp, n_proj):
     from load_balancing_planner_b200 import moonep
