@@ -83,18 +83,26 @@ KERNELS_PER_STEP = 3
 PAGES_POINTS = (10.0, 20.0)
 
 
+def copy_source_hash():
+    """Hash of the sources of the copy kernels (copy.cu and the shared header)."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in ("copy.cu", "moonep_internal.cuh"):
+        with open(os.path.join(ROOT, "load_balancing_planner_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
 def recorded_traffic(kernel):
     """DRAM bytes per launch of `kernel` at the training shape, from the ncu
     record in profiles/dram_traffic_train.md -- only if that record was taken
     on the current source of the copy kernels (hash match), else None."""
-    import hashlib
     import re
     try:
-        with open(os.path.join(ROOT, "load_balancing_planner_b200", "csrc", "copy.cu"), "rb") as f:
-            sha = hashlib.sha256(f.read()).hexdigest()[:16]
+        sha = copy_source_hash()
         with open(os.path.join(ROOT, "profiles", "dram_traffic_train.md")) as f:
             for line in f:
-                m = re.search(r"traffic: kernel=(\w+) bytes_per_launch=(\d+) copy_cu_sha256=(\w+)", line)
+                m = re.search(r"traffic: kernel=(\w+) bytes_per_launch=(\d+) copy_src_sha256=(\w+)", line)
                 if m and m.group(1) == kernel and m.group(3) == sha:
                     return int(m.group(2))
     except OSError:
