@@ -678,13 +678,41 @@ def oracle_sample(w, routes_np, ranks_sampled, seed):
     return total_b, total_s
 
 
+def oracle_weight_legs(seed, H=7168, Hp=2048, experts=2):
+    """The oracle's prefetch and reduce_grad on one host core, on a sample of
+    the inference / backward legs: `experts` expert matrices [H, H'], each
+    copied to two slots (prefetch) or summed from two slots (reduce_grad).
+    Returns {leg: GB/s} over the legs' algorithmic bytes."""
+    import oracle
+    hhp = H * Hp
+    g = np.random.default_rng(seed)
+    se = np.full((2, experts), -1, np.int32)
+    se[0, :] = np.arange(experts)
+    se[1, :] = np.arange(experts)  # two holders per expert
+    W = g.integers(0, 1 << 16, size=(experts, hhp), dtype=np.uint16)
+    pool = np.zeros((2 * experts, hhp), np.uint16)
+    t0 = time.perf_counter()
+    oracle.prefetch(se, W, pool)
+    t_pf = time.perf_counter() - t0
+    G = g.standard_normal((experts, hhp), dtype=np.float32)
+    RB = g.standard_normal((2 * experts, hhp), dtype=np.float32)
+    t0 = time.perf_counter()
+    oracle.reduce_grad(se, G, RB)
+    t_rg = time.perf_counter() - t0
+    d, u = experts, 2 * experts
+    return {"prefetch_weight_gbs": round((d + u) * hhp * 2 / t_pf / 1e9, 3),
+            "reduce_grad_gbs": round((2 * d + 2 * u) * hhp * 4 / t_rg / 1e9, 3),
+            "sample": f"{experts} expert matrices [{H}, {Hp}], two slots each"}
+
+
 def cpu_baseline(w, routes, seed):
     ranks = 4
     b, s = oracle_sample(w, [r["topk_np"] for r in routes], ranks, seed)
     return {"value": round(b / s / 1e9, 3), "unit": "GB/s", "cores": 1, "kind": "oracle",
             "sample": f"full plan of each of the {len(routes)} routings (all {w['R']} ranks) + dispatch and "
                       f"combine of every token of {ranks} of {w['R']} source ranks, single-threaded C, "
-                      f"{s:.1f} s", "host_cores_available": os.cpu_count()}
+                      f"{s:.1f} s", "host_cores_available": os.cpu_count(),
+            "legs": oracle_weight_legs(seed)}
 
 
 # ---------------------------------------------------------------- reference arm

@@ -30,6 +30,9 @@ CASES = [
     ("max_e", 8, 300, 8, 4096, 512, 16, 0, "hot8", [2.0]),
     ("k32", 2, 100, 32, 64, 32, 4, 0, "zipf", [0.5]),
     ("many_ranks", 64, 40, 4, 256, 4, 8, 0, "hot8", [3.0]),
+    # 16384 tokens per rank: chunks grow until every block is resident, and
+    # each block reads many earlier chunk rows of its rank
+    ("long_seq", 8, 16384, 8, 256, 32, 128, 0, "hot8", [2.0]),
 ]
 
 
