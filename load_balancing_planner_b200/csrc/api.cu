@@ -169,7 +169,7 @@ extern "C" int moonep_create(const moonep_config_t *cfg, moonep_handle_t *out) {
     h->grid_combine = h->sms * combine_blocks_per_sm(d.K);
     h->grid_weights = h->sms * weights_blocks_per_sm();
 
-    const size_t wsb = workspace_bytes(d);
+    const size_t wsb = (workspace_bytes(d) + 255) / 256 * 256 + sizeof(int32_t) * (size_t)d.R * gemm_pair_slots(d);
     if ((e = cudaMalloc(&h->ws_mem, wsb)) != cudaSuccess) { free(h); return fail_cuda(e); }
     if ((e = cudaMemset(h->ws_mem, 0, wsb)) != cudaSuccess) {
         cudaFree(h->ws_mem);
@@ -303,7 +303,8 @@ extern "C" int moonep_group_gemm(moonep_handle_t h, const moonep_plan_t *plan, c
         return MOONEP_ERR_ALIGN;
     const int rc = gemm_supported(h->d, Hp);
     if (rc != MOONEP_OK) return rc;
-    return launch_group_gemm(h->d, plan, x_nvs, weights, pool, y_nvs, Hp, reinterpret_cast<cudaStream_t>(stream));
+    int32_t *pairs = reinterpret_cast<int32_t *>(static_cast<char *>(h->ws_mem) + (workspace_bytes(h->d) + 255) / 256 * 256);
+    return launch_group_gemm(h->d, plan, x_nvs, weights, pool, y_nvs, Hp, pairs, reinterpret_cast<cudaStream_t>(stream));
 }
 
 extern "C" int moonep_read_status(const moonep_plan_t *plan, int32_t *status, moonep_stream_t stream) {

@@ -7,40 +7,35 @@
 // Wrow = W[i] for i < E (home rows, and inference overflow rows read from the
 // home expert), pool[r][i - E] for slot rows.
 //
-// sm_100a design: one CTA per 128 x 256 output tile.  Warp 0 streams A (the
-// tile's 128 buffer rows) and B (the row's weight) through a 4-stage ring in
-// shared memory with TMA, 128-byte swizzled; warp 1 issues tcgen05.mma
-// (bf16 x bf16 -> fp32, M=128, N=256, K=16) into a 256-column accumulator in
-// tensor memory and frees each stage with tcgen05.commit; then all four warps
-// read the accumulator back (tcgen05.ld, one warp per 32 lanes), round to
-// bf16 and store.  Rows are 128-aligned inside their segments because the
-// padding unit token_padding is a multiple of 128, so a tile never straddles
-// two weight rows.  Every mbarrier wait is bounded; a timeout sets
-// MOONEP_STATUS_TIMEOUT and the CTA drains what it issued before it frees the
-// tensor memory.
+// sm_100a design: a cluster of two CTAs (one per SM) computes a 256 x 256
+// output tile with tcgen05.mma.cta_group::2 (bf16 x bf16 -> fp32, M=256,
+// N=256, K=16).  Each CTA holds 128 rows of A and 128 of the 256 columns of
+// B in shared memory, so an SM reads 16 KB of operands per MMA instead of the
+// 24 KB a one-SM 128 x 256 tile needs; the one-SM design was bound by shared
+// memory bandwidth (operand reads plus TMA fills) at about 70 % of the bf16
+// peak.  Warp 0 of each CTA streams its halves through a 6-stage ring with
+// 2-D TMA loads (128-byte swizzle, no multicast) that complete on the pair
+// leader's mbarriers; one thread of the leader issues the MMAs into a
+// 256-column accumulator in each CTA's tensor memory, and its commits free
+// the stages and signal the accumulators in both CTAs; all four warps of each
+// CTA read their 128 rows back (tcgen05.ld), round to bf16 and store.
+//
+// Tiles: rows are padded to token_padding, a multiple of 128, so every
+// 128-row tile lies in one plan row; pair_map_kernel pairs consecutive tiles
+// of the same plan row, so both halves of a pair share one weight, and an odd
+// tile count leaves a dead second half that is computed on valid rows and not
+// stored.  Every mbarrier wait is bounded; a timeout sets
+// MOONEP_STATUS_TIMEOUT.
 #include <cuda.h>
 
 #include "moonep_internal.cuh"
 
 namespace moonep {
 
-constexpr int kGBM = 128, kGBN = 256, kGBK = 64, kGStages = 4;
+constexpr int kGBM = 128, kGBN = 256, kGBK = 64;  // per-CTA rows, tile columns, K per stage
 constexpr int kGThreads = 128;
-constexpr int kGTileA = kGBM * kGBK * 2;     // 16 KB
-constexpr int kGTileB = kGBK * kGBN * 2;     // 32 KB: 4 boxes of 64 K-rows x 64 columns
-constexpr int kGBoxB = kGBK * 64 * 2;        // 8 KB
-constexpr uint32_t kGPolls = 1u << 22;       // bounded mbarrier waits (try_wait suspends between polls)
-constexpr int kGSmem = 1024 + kGStages * (kGTileA + kGTileB) + 256;
-
-struct GemmArgs {
-    CUtensorMap tx;  // x [R*NvS, H], box {64, 128}
-    CUtensorMap tw;  // W [E*H, Hp], box {64, 64}
-    CUtensorMap tp;  // pool [R*B*H, Hp], box {64, 64} (== tw when B == 0)
-    const int32_t *cu_seqlens;  // [R, E+B]
-    int32_t *status;            // plan status: read, TIMEOUT OR-ed in
-    void *y;                    // [R*NvS, Hp] bf16
-    int E, B, H, Hp, nvs, NR, mtiles;
-};
+constexpr int kGBoxB = kGBK * 64 * 2;              // 8 KB: one TMA box of B (64 K-rows x 64 columns)
+constexpr uint32_t kGPolls = 1u << 22;             // bounded mbarrier waits (try_wait suspends between polls)
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -73,15 +68,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
     return false;
 }
 
-// 2-D TMA tile load into this CTA's shared memory, completion on `bar`.
-__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int c0, int c1, uint64_t *bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
-            smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
-        : "memory");
-}
-
 // Shared-memory matrix descriptors (tcgen05), 128-byte swizzle, version 1.
 // A: K-major rows of 128 bytes, 8-row groups 1024 bytes apart.
 __device__ __forceinline__ uint64_t desc_k_sw128(uint32_t saddr) {
@@ -95,28 +81,103 @@ __device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t saddr) {
            ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
-// kind::f16 instruction descriptor: D fp32, A and B bf16, A K-major, B
-// N-major, N = 256, M = 128.
-constexpr uint32_t kGIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((uint32_t)(kGBN >> 3) << 17) |
-                             ((uint32_t)(kGBM >> 4) << 24);
 
-__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+constexpr int kGStages = 6;
+constexpr int kGTileA = kGBM * kGBK * 2;        // 16 KB: this CTA's 128 rows
+constexpr int kGTileB = kGBK * (kGBN / 2) * 2;  // 16 KB: this CTA's 128 columns (2 boxes)
+constexpr int kGSmem = 1024 + kGStages * (kGTileA + kGTileB) + 256;
+constexpr uint32_t kGIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((uint32_t)(kGBN >> 3) << 17) |
+                              ((uint32_t)(256 >> 4) << 24);
+
+struct GemmArgs {
+    CUtensorMap tx, tw, tp;
+    const int32_t *cu_seqlens;  // [R, E+B]
+    const int32_t *pairs;       // [R, pmax]: (plan row << 12) | pair index in the row, or -1
+    int32_t *status;
+    void *y;
+    int R, E, B, H, Hp, nvs, NR, pmax, ntiles;
+};
+
+// pairs[r][q]: the q-th 256-row pair of rank r, in plan-row order; -1 past
+// the last pair, and everywhere for a failed plan.
+__global__ void __launch_bounds__(256) pair_map_kernel(const int32_t *cu_seqlens, const int32_t *status,
+                                                        int32_t *pairs, int NR, int pmax) {
+    pdl_wait();
+    const int r = blockIdx.x, tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    __shared__ int s_warp[8], s_carry;
+    const int32_t *cu = cu_seqlens + (int64_t)r * NR;
+    int32_t *out = pairs + (int64_t)r * pmax;
+    const bool failed = ld_cg(status) != 0;
+    if (tid == 0) s_carry = 0;
+    __syncthreads();
+    for (int i0 = 0; i0 < NR && !failed; i0 += 256) {
+        const int i = i0 + tid;
+        int np = 0;
+        if (i < NR) {
+            const int lp = ld_cg(cu + i) - (i > 0 ? ld_cg(cu + i - 1) : 0);  // padded rows, a multiple of 128
+            np = (lp / kGBM + 1) / 2;
+        }
+        int incl = np;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        if (lane == 31) s_warp[w] = incl;
+        __syncthreads();
+        int before = s_carry;
+        for (int k = 0; k < w; ++k) before += s_warp[k];
+        const int first = before + incl - np;
+        for (int j = 0; j < np; ++j)
+            if (first + j < pmax) out[first + j] = (i << 12) | j;
+        __syncthreads();
+        if (tid == 0)
+            for (int k = 0; k < 8; ++k) s_carry += s_warp[k];
+        __syncthreads();
+    }
+    const int used = failed ? 0 : s_carry;
+    for (int q = used + tid; q < pmax; q += 256) out[q] = -1;
+}
+
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+    uint32_t out;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(addr), "r"(rank));
+    return out;
+}
+
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map, int c0, int c1,
+                                                 uint32_t bar_cluster) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+        "%3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar_cluster)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_bf16_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
         "l"(adesc), "l"(bdesc), "r"(kGIdesc), "r"(accumulate)
         : "memory");
 }
 
-__device__ __forceinline__ void umma_commit(uint64_t *bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-                 : "memory");
+__device__ __forceinline__ void umma_commit_pair(uint64_t *bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"((uint16_t)3)
+        : "memory");
 }
 
-__global__ void __launch_bounds__(kGThreads, 1) group_gemm_kernel(const __grid_constant__ GemmArgs a) {
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
+    group_gemm_kernel(const __grid_constant__ GemmArgs a) {
     extern __shared__ uint8_t gsm_raw[];
-    // 1024-byte alignment for the swizzled tiles
     uint8_t *gsm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(gsm_raw) + 1023) & ~(uintptr_t)1023);
     uint8_t *sA = gsm;
     uint8_t *sB = gsm + kGStages * kGTileA;
@@ -124,28 +185,37 @@ __global__ void __launch_bounds__(kGThreads, 1) group_gemm_kernel(const __grid_c
     uint64_t *empty = full + kGStages;
     uint64_t *accum = empty + kGStages;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accum + 1);
-    __shared__ int s_row, s_err;
+    __shared__ int s_v, s_start, s_lp, s_err;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int nt = blockIdx.x;
-    const int r = blockIdx.y / a.mtiles, row0 = (blockIdx.y - r * a.mtiles) * kGBM;
+    uint32_t crank;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(crank));
+    const int c = blockIdx.x >> 1;
+    const int nt = c % a.ntiles, rq = c / a.ntiles;
+    const int r = rq / a.pmax, q = rq - r * a.pmax;
 
     pdl_wait();
-    // the weight row of this tile: the first row i whose inclusive end
-    // cu_seqlens[r][i] lies past row0 (none: the tile is past the used rows;
-    // a failed plan: nothing to compute)
+    // The pair table is written before this kernel and read only here, so
+    // both CTAs of a pair take the same decision.
     if (tid == 0) {
-        s_row = ld_cg(a.status) != 0 ? -1 : a.NR;
+        const int v = ld_cg(a.pairs + (int64_t)r * a.pmax + q);
+        s_v = v;
         s_err = 0;
+        if (v >= 0) {
+            const int i = v >> 12;
+            const int32_t *cu = a.cu_seqlens + (int64_t)r * a.NR;
+            const int end = ld_cg(cu + i), beg = i > 0 ? ld_cg(cu + i - 1) : 0;
+            s_start = beg;
+            s_lp = end - beg;
+        }
     }
     __syncthreads();
-    const int32_t *cu = a.cu_seqlens + (int64_t)r * a.NR;
-    if (s_row >= 0)
-        for (int i = tid; i < a.NR; i += kGThreads)
-            if (ld_cg(cu + i) > row0) atomicMin(&s_row, i);
-    __syncthreads();
-    const int wrow = s_row;
-    if (wrow < 0 || wrow >= a.NR) return;  // uniform over the block
+    const int v = s_v;
+    if (v < 0) return;  // both CTAs of the pair
+    const int wrow = v >> 12, pj = v & 4095;
+    const int off = 2 * kGBM * pj + kGBM * (int)crank;
+    const bool live = off < s_lp;
+    const int row0 = s_start + (live ? off : 2 * kGBM * pj);
     const CUtensorMap *tb = wrow < a.E ? &a.tw : &a.tp;
     const int brow0 = (wrow < a.E ? wrow : r * a.B + (wrow - a.E)) * a.H;
 
@@ -158,97 +228,92 @@ __global__ void __launch_bounds__(kGThreads, 1) group_gemm_kernel(const __grid_c
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 0) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                      "r"(kGBN));
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-    __syncthreads();
+    cluster_sync();  // both CTAs' barriers are initialised before either signals the other
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const uint32_t tmem = *tmem_slot;
     const int nk = a.H / kGBK;
+    volatile int *err = &s_err;
 
     if (warp == 0 && lane == 0) {
-        // producer
-        int issued = 0;
         for (int kb = 0; kb < nk; ++kb) {
             const int s = kb % kGStages;
             if (kb >= kGStages && !mbar_wait(&empty[s], ((kb / kGStages) - 1) & 1)) {
                 atomicOr(a.status, MOONEP_STATUS_TIMEOUT);
-                s_err = 1;
+                *err = 1;
                 break;
             }
-            if (*(volatile int *)&s_err) break;
-            mbar_expect_tx(&full[s], kGTileA + kGTileB);
-            tma_load_2d(sA + s * kGTileA, &a.tx, kb * kGBK, r * a.nvs + row0, &full[s]);
+            const uint32_t bar = mapa_shared(smem_u32(&full[s]), 0);  // the leader's barrier
+            if (crank == 0) mbar_expect_tx(&full[s], 2 * (kGTileA + kGTileB));
+            tma_load_2d_pair(smem_u32(sA + s * kGTileA), &a.tx, kb * kGBK, r * a.nvs + row0, bar);
 #pragma unroll
-            for (int q = 0; q < kGBN / 64; ++q)
-                tma_load_2d(sB + s * kGTileB + q * kGBoxB, tb, nt * kGBN + q * 64, brow0 + kb * kGBK, &full[s]);
-            issued = kb + 1;
+            for (int qb = 0; qb < 2; ++qb)
+                tma_load_2d_pair(smem_u32(sB + s * kGTileB + qb * kGBoxB), tb,
+                                 nt * kGBN + (int)crank * (kGBN / 2) + qb * 64, brow0 + kb * kGBK, bar);
         }
-        // the last load issued into each stage has landed before anyone leaves
-        for (int kb = max(0, issued - kGStages); kb < issued; ++kb)
-            if (!mbar_wait(&full[kb % kGStages], (kb / kGStages) & 1)) atomicOr(a.status, MOONEP_STATUS_TIMEOUT);
-    } else if (warp == 1 && lane == 0) {
-        // MMA issuer
+    } else if (warp == 1 && lane == 0 && crank == 0) {
         for (int kb = 0; kb < nk; ++kb) {
             const int s = kb % kGStages;
             if (!mbar_wait(&full[s], (kb / kGStages) & 1)) {
                 atomicOr(a.status, MOONEP_STATUS_TIMEOUT);
-                s_err = 1;
+                *err = 1;
                 break;
             }
-            if (*(volatile int *)&s_err) break;
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
             const uint32_t a0 = smem_u32(sA + s * kGTileA), b0 = smem_u32(sB + s * kGTileB);
 #pragma unroll
             for (int k = 0; k < kGBK / 16; ++k)
-                umma_bf16(tmem, desc_k_sw128(a0 + k * 32), desc_mn_sw128(b0 + k * 16 * 128), (kb | k) != 0);
-            umma_commit(&empty[s]);  // the stage is free once these MMAs have read it
+                umma_bf16_pair(tmem, desc_k_sw128(a0 + k * 32), desc_mn_sw128(b0 + k * 16 * 128), (kb | k) != 0);
+            umma_commit_pair(&empty[s]);  // frees stage s in both CTAs once these MMAs have read it
         }
-        umma_commit(accum);  // every MMA issued above has completed
+        umma_commit_pair(accum);  // both CTAs' accumulators are complete
     }
     __syncwarp();
 
-    // epilogue: warp w owns accumulator lanes (tile rows) 32w .. 32w+31
-    const bool ok = __all_sync(0xffffffffu, mbar_wait(accum, 0));  // warp-uniform: tcgen05.ld is .aligned
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(accum, 0));
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     if (!ok) {
         if (lane == 0) atomicOr(a.status, MOONEP_STATUS_TIMEOUT);
-    } else if (!*(volatile int *)&s_err) {
+    } else if (live && !*err) {
         const int row = row0 + warp * 32 + lane;
         uint4 *yrow = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.y) +
                                                 ((int64_t)r * a.nvs + row) * a.Hp + nt * kGBN);
 #pragma unroll 1
-        for (int c = 0; c < kGBN / 32; ++c) {
-            uint32_t v[32];
-            const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + c * 32;
+        for (int cc = 0; cc < kGBN / 32; ++cc) {
+            uint32_t v32[32];
+            const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + cc * 32;
             asm volatile(
                 "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
                 "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-                : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-                  "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
-                  "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]),
-                  "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]),
-                  "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+                : "=r"(v32[0]), "=r"(v32[1]), "=r"(v32[2]), "=r"(v32[3]), "=r"(v32[4]), "=r"(v32[5]), "=r"(v32[6]),
+                  "=r"(v32[7]), "=r"(v32[8]), "=r"(v32[9]), "=r"(v32[10]), "=r"(v32[11]), "=r"(v32[12]),
+                  "=r"(v32[13]), "=r"(v32[14]), "=r"(v32[15]), "=r"(v32[16]), "=r"(v32[17]), "=r"(v32[18]),
+                  "=r"(v32[19]), "=r"(v32[20]), "=r"(v32[21]), "=r"(v32[22]), "=r"(v32[23]), "=r"(v32[24]),
+                  "=r"(v32[25]), "=r"(v32[26]), "=r"(v32[27]), "=r"(v32[28]), "=r"(v32[29]), "=r"(v32[30]),
+                  "=r"(v32[31])
                 : "r"(taddr));
             asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-            uint32_t p[16];
+            uint32_t pk[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-                const __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
-                p[j] = *reinterpret_cast<const uint32_t *>(&h2);
+                const __nv_bfloat162 h2 =
+                    __floats2bfloat162_rn(__uint_as_float(v32[2 * j]), __uint_as_float(v32[2 * j + 1]));
+                pk[j] = *reinterpret_cast<const uint32_t *>(&h2);
             }
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-                yrow[c * 4 + j] = make_uint4(p[4 * j], p[4 * j + 1], p[4 * j + 2], p[4 * j + 3]);
+                yrow[cc * 4 + j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
         }
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-    __syncthreads();
+    cluster_sync();  // neither CTA frees its memory while the pair's MMAs may still read it
     if (warp == 0) {
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kGBN));
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kGBN));
     }
 }
 
@@ -298,7 +363,7 @@ cudaError_t gemm_set_smem_limit() {
 }
 
 int launch_group_gemm(const Dims &d, const moonep_plan_t *plan, const void *x, const void *W, const void *pool,
-                      void *y, int64_t Hp, cudaStream_t st) {
+                      void *y, int64_t Hp, int32_t *pairs, cudaStream_t st) {
     GemmArgs a;
     memset(&a, 0, sizeof(a));
     if (!make_map(&a.tx, x, (uint64_t)d.R * d.nvs, d.H, kGBM) ||
@@ -306,17 +371,23 @@ int launch_group_gemm(const Dims &d, const moonep_plan_t *plan, const void *x, c
         !make_map(&a.tp, d.B > 0 ? pool : W, d.B > 0 ? (uint64_t)d.R * d.B * d.H : (uint64_t)d.E * d.H, Hp, kGBK))
         return MOONEP_ERR_CUDA;
     a.cu_seqlens = plan->cu_seqlens;
+    a.pairs = pairs;
     a.status = plan->status;
     a.y = y;
+    a.R = d.R;
     a.E = d.E;
     a.B = d.B;
     a.H = d.H;
     a.Hp = (int)Hp;
     a.nvs = d.nvs;
     a.NR = d.NR;
-    a.mtiles = d.nvs / kGBM;
+    a.pmax = gemm_pair_slots(d);
+    a.ntiles = (int)(Hp / kGBN);
+    pair_map_kernel<<<d.R, 256, 0, st>>>(plan->cu_seqlens, plan->status, pairs, d.NR, a.pmax);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail_cuda(e);
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(Hp / kGBN), (unsigned)(d.R * a.mtiles));
+    cfg.gridDim = dim3((unsigned)(2 * (int64_t)d.R * a.pmax * a.ntiles));
     cfg.blockDim = dim3(kGThreads);
     cfg.dynamicSmemBytes = kGSmem;
     cfg.stream = st;
@@ -325,8 +396,10 @@ int launch_group_gemm(const Dims &d, const moonep_plan_t *plan, const void *x, c
     at[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, group_gemm_kernel, a);
+    e = cudaLaunchKernelEx(&cfg, group_gemm_kernel, a);
     return e == cudaSuccess ? MOONEP_OK : fail_cuda(e);
 }
+
+int gemm_pair_slots(const Dims &d) { return (d.nvs / kGBM + d.NR + 1) / 2; }
 
 }  // namespace moonep

@@ -91,7 +91,8 @@ int weights_blocks_per_sm();
 int gemm_supported(const Dims &d, int64_t Hp);
 cudaError_t gemm_set_smem_limit();
 int launch_group_gemm(const Dims &d, const moonep_plan_t *plan, const void *x, const void *W, const void *pool,
-                      void *y, int64_t Hp, cudaStream_t st);
+                      void *y, int64_t Hp, int32_t *pairs, cudaStream_t st);
+int gemm_pair_slots(const Dims &d);
 
 // ---- host helpers shared by the entry points (api.cu) ----------------------
 int fail_cuda(cudaError_t e);                  // records the error text, returns MOONEP_ERR_CUDA
