@@ -84,10 +84,10 @@ PAGES_POINTS = (10.0, 20.0)
 
 
 def copy_source_hash():
-    """Hash of the sources of the copy kernels (copy.cu and the shared header)."""
+    """Hash of the sources of the copy kernels (copy.cu and the bulk-copy helpers)."""
     import hashlib
     h = hashlib.sha256()
-    for name in ("copy.cu", "moonep_internal.cuh"):
+    for name in ("copy.cu", "bulk.cuh"):
         with open(os.path.join(ROOT, "load_balancing_planner_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
