@@ -102,3 +102,38 @@ def test_wide_plan_many_short_rows(cuda):
     # nearly every tile pair has a dead second half
     got = _run(R=8, S=256, K=8, E=1024, B=128, H=128, Hp=256, mode=0, mv=2.0, profile="hot8", seed=45)
     assert got["cu_seqlens"].size > 6144
+
+
+def test_training_shape_sampled(cuda):
+    # R=8, S=4096, K=8, E=256, B=32, H=7168, H'=2048 at maxvio 2, in the launch
+    # configuration the bench times: 512 sampled real slots (home and slot
+    # rows) x 64 sampled columns against fp64 dot products
+    from load_balancing_planner_b200 import moonep
+    R, S, K, E, B, H, Hp, tp = 8, 4096, 8, 256, 32, 7168, 2048, 128
+    tk, tpe, _ = problem(R, S, K, E, 2.0, "hot8", seed=46)
+    h = moonep.moonep_create(S, H, K, E, R, B, tp)
+    p = gpu_plan(h, tk, tpe)
+    x = synth.hidden_bf16(R, S, H, seed=46).cuda()
+    buf, _ = moonep.moonep_dispatch(h, p, x)
+    g = torch.Generator(device="cuda").manual_seed(46)
+    W = (torch.randn((E, H, Hp), generator=g, device="cuda") * H ** -0.5).to(torch.bfloat16)
+    pool = torch.empty((R, B, H, Hp), dtype=torch.bfloat16, device="cuda")
+    moonep.moonep_prefetch_weight(h, p, [W], [pool])
+    y = moonep.moonep_group_gemm(h, p, buf, W, pool)
+    torch.cuda.synchronize()
+    assert moonep.moonep_read_status(p) == 0
+    got = plan_to_numpy(p)
+    segs = oracle.segments(got["cu_seqlens"], got["row_counts"], E, tp)
+    rng = np.random.default_rng(0)
+    slot_segs = [sg for sg in segs if sg[3] >= E]
+    assert slot_segs
+    picks = [segs[i] for i in rng.integers(0, len(segs), 448)] + [slot_segs[i] for i in rng.integers(0, len(slot_segs), 64)]
+    cols = torch.from_numpy(np.sort(rng.choice(Hp, 64, replace=False))).cuda()
+    for r, s0, n, i in picks:
+        row = s0 + int(rng.integers(0, n))
+        w = (W[i] if i < E else pool[r, i - E])[:, cols].double().cpu().numpy()
+        xr = buf[r, row].double().cpu().numpy()
+        want = xr @ w
+        have = y[r, row, cols].double().cpu().numpy()
+        assert rel_close(have, want, 1e-2).all(), (r, row, i)
+    h.close()
