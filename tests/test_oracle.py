@@ -183,6 +183,34 @@ def test_inference_slots_by_count_and_by_id():
         assert np.array_equal(q1[k], q2[k]), k
 
 
+@pytest.mark.parametrize("rank1,slot1,slot2", [
+    # e2 and e3 each give 2 picks: both rules take e2 (a tie goes to the lower id)
+    ([2, 2, 3, 3, 4, 5, 6, 7], 2, 2),
+    # e2 gives 1 pick, e3 gives 3: by id e2, by count e3
+    ([2, 3, 3, 3, 4, 5, 6, 7], 2, 3),
+])
+def test_inference_slot_choice_worked_example(rank1, slot1, slot2):
+    # Worked by hand.  R=2, E=8 (G=4), S=8, K=1, B=1, token_padding=1.
+    # Rank 0 picks e0 x4, e1 x4; rank 1 picks rank1.  Group 0's sequence is
+    # e0[0,4) e1[4,8) then e2, e3: L_0 = 12, L_1 = 4, C = 8, so rank 1 takes
+    # the last 4 picks of group 0, i.e. all of e2's and e3's.  With one slot,
+    # the expert not taken stays on rank 1's overflow home row.
+    tk = np.array([[0] * 4 + [1] * 4, rank1], np.int32).reshape(2, 8, 1)
+    n2, n3 = rank1.count(2), rank1.count(3)
+    for mode, slot in ((1, slot1), (2, slot2)):
+        p = oracle.plan(tk, 8, 1, 1, mode)
+        assert p["status"] == 0
+        assert p["assign"].tolist() == [[8, -1, 0, 0], [4, 0, 8, 4]]
+        assert p["slot_expert"].tolist() == [[-1], [slot]]
+        ovf = 5 - slot  # the other of e2, e3
+        want = [0] * 9
+        want[ovf] = n2 if ovf == 2 else n3
+        want[4:8] = [1, 1, 1, 1]
+        want[8] = n2 if slot == 2 else n3
+        assert p["row_counts"][1].tolist() == want
+        assert p["row_counts"][0].tolist() == [4, 4, 0, 0, 0, 0, 0, 0, 0]
+
+
 # ------------------------------------------------ special cases: stable sort
 def _sorted_layout(tk, E, B, tp, h, G):
     """Where rank h's picks go when no copies are made: a stable argsort by
