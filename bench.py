@@ -407,6 +407,7 @@ def run_ours(args, world, rank, local):
             result["legs"]["pages_maxvio_points"] = run_pages_points(w, seed, dev, h, plan, hidden, weights,
                                                                      buf, wn, out, gw, stream)
             result["legs"]["group_gemm"] = run_group_gemm_leg(dev, seed)
+            result["legs"]["rank_local"] = run_rank_local_leg(w, seed, dev, hidden, weights, routes, stream)
     if not args.no_e2e:
         result["e2e"] = run_e2e(args, h, plan, w, routes, dev, stream, world)
     h.close()
@@ -447,6 +448,57 @@ def run_pages_points(w, seed, dev, h, plan, hidden, weights, buf, wn, out, gw, s
                               dc_gbs=round((db + cb) / (dc * 1e-3) / 1e9, 1),
                               used_slots=int((plan.slots() >= 0).sum().item()))
     return pts
+
+
+def run_rank_local_leg(w, seed, dev, hidden, weights, routes, stream, reps=10):
+    """The layer in its per-rank form, as each GPU of a real EP group runs
+    it: moonep_plan_rank from the rank's own picks and the gathered counts,
+    then moonep_dispatch_rank / moonep_combine_rank through a table of the R
+    ranks' buffers (R separate allocations here).  The R ranks' launches run
+    back to back on this GPU; bytes and routing are the headline step's."""
+    import torch
+    from load_balancing_planner_b200 import moonep
+    R, S, K, E, B, H, tp = w["R"], w["S"], w["K"], w["E"], w["B"], w["H"], w["tp"]
+    h = moonep.moonep_create(S, H, K, E, R, B, tp, mode=w["mode"])
+    nvs = h.nvs
+    bufs = [torch.empty((nvs, H), dtype=torch.bfloat16, device=dev) for _ in range(R)]
+    wbufs = [torch.empty((nvs,), dtype=torch.float32, device=dev) for _ in range(R)]
+    out = torch.empty((R, S, H), dtype=torch.bfloat16, device=dev)
+    gw = torch.empty((R, S, K), dtype=torch.float32, device=dev)
+    plans = [moonep.Plan(h, dev, rank=r) for r in range(R)]
+    db, cb = dc_bytes(R, S, K, H)
+    res = {}
+    for rt in routes:
+        if rt["target"] not in (0.0, 2.0):
+            continue
+        topk = [rt["topk"][r].contiguous() for r in range(R)]
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(reps + 3)]
+        for e in evs:
+            e[0].record(stream)
+            for r in range(R):
+                moonep.moonep_plan_rank(h, r, topk[r], rt["tpe"], plans[r])
+            e[1].record(stream)
+            for r in range(R):
+                moonep.moonep_dispatch_rank(h, plans[r], hidden[r], weights[r], bufs, wbufs)
+            e[2].record(stream)
+            for r in range(R):
+                moonep.moonep_combine_rank(h, plans[r], bufs, wbufs, out[r], gw[r])
+            e[3].record(stream)
+        torch.cuda.synchronize()
+        if any(moonep.moonep_read_status(p) != 0 for p in plans):
+            raise RuntimeError("rank plan status")
+        evs = evs[3:]
+        dc = statistics.median([e[1].elapsed_time(e[3]) for e in evs])
+        res[f"{rt['target']:g}"] = dict(
+            planner_us_per_rank=round(statistics.median([e[0].elapsed_time(e[1]) for e in evs]) * 1e3 / R, 2),
+            dispatch_us=round(statistics.median([e[1].elapsed_time(e[2]) for e in evs]) * 1e3, 1),
+            combine_us=round(statistics.median([e[2].elapsed_time(e[3]) for e in evs]) * 1e3, 1),
+            dc_gbs=round((db + cb) / (dc * 1e-3) / 1e9, 1))
+    h.close()
+    return dict(workload=describe(w) + "; per-rank calls of all R ranks, buffers as R allocations",
+                planner="R rank plans back to back per layer, reported per rank (each GPU of a real group "
+                        "plans only its own share, concurrently)",
+                points=res)
 
 
 def run_group_gemm_leg(dev, seed, mv=2.0, Hp=2048, reps=10, config="train"):

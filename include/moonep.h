@@ -234,6 +234,73 @@ MOONEP_API int moonep_group_gemm(moonep_handle_t h, const moonep_plan_t *plan, c
                                  moonep_stream_t stream);
 
 /*
+ * ---- One rank of a real EP group ----
+ *
+ * On R GPUs each rank holds only its own router output, and the R dispatched
+ * buffers live on R devices.  README "dispatch fwd" gives every rank its
+ * local tokens_per_expert [E]; gathered from all ranks (an all-gather of
+ * R*E int32, which the caller runs, e.g. with NCCL), they are all the
+ * planner needs besides the rank's own picks: every rank then derives the
+ * same layout, and each writes dst for its own picks only.  Dispatch and
+ * combine take the R ranks' buffers as a table of device pointers (peer
+ * mappings of the other ranks' memory on a real group; R separate
+ * allocations on one GPU).  The slot encoding is the group one: dst =
+ * q*NvS + i is row i of rank q's buffer.  The calls share the handle's
+ * conventions; moonep_plan_rank has its own planning workspace in the
+ * handle, so it may alternate with moonep_plan on one stream.
+ */
+
+/*
+ * Plan rank `rank`'s share of one layer.
+ *   topk        [S,K] int32  the rank's own picks
+ *   counts_all  [R,E] int32  every rank's router counts, row q = rank q's
+ *                            tokens_per_expert (the gathered table)
+ *   plan        as for moonep_plan, except dst: [S,K], the slots of this
+ *               rank's picks.  cu_seqlens, row_counts, slot_expert, assign
+ *               and maxvio hold the whole group's layout (identical on every
+ *               rank, and equal to moonep_plan's for the same routing);
+ *               counts is a copy of counts_all.
+ * Result: equal to the rank's slice of moonep_plan's plan for the group's
+ * picks.  Device-side errors: BAD_EXPERT and DUP_EXPERT in the rank's picks;
+ * COUNT_MISMATCH when row `rank` of counts_all differs from the picks, or
+ * when any row holds a negative count or does not sum to S*K (then the other
+ * plan arrays are unspecified).  A rank sees only its own picks: a group is consistent
+ * when every rank's status is 0 (combine them, e.g. with an all-reduce).
+ * ERR_SIZE when rank is outside [0, R).
+ */
+MOONEP_API int moonep_plan_rank(moonep_handle_t h, int32_t rank, const int32_t *topk, const int32_t *counts_all,
+                                const moonep_plan_t *plan, moonep_stream_t stream);
+
+/*
+ * Dispatch of one rank's tokens with a plan from moonep_plan_rank: every row
+ * goes straight to its K slots in the destination ranks' buffers.
+ *   hidden            [S,H] bf16   the rank's token rows (16-byte aligned)
+ *   route_weights     [S,K] fp32   or NULL
+ *   hidden_nvs        R device pointers (host array): rank q's [NvS,H] bf16
+ *                     buffer, each 16-byte aligned; written at real slots only
+ *   route_weights_nvs R device pointers to rank q's [NvS] fp32, or NULL; with
+ *                     route_weights given, written at the real slots
+ * The tables are read on the host at the call; the buffers they name must
+ * stay valid until the launch completes.
+ */
+MOONEP_API int moonep_dispatch_rank(moonep_handle_t h, const moonep_plan_t *plan, const void *hidden,
+                                    const float *route_weights, void *const *hidden_nvs,
+                                    float *const *route_weights_nvs, moonep_stream_t stream);
+
+/*
+ * Combine of one rank's tokens with a plan from moonep_plan_rank:
+ * out[t,:] = bf16(sum_k w_k * y[dst[t,k]]) in fp32, k order, as moonep_combine.
+ *   hidden_nvs        R device pointers: rank q's expert output [NvS,H] bf16
+ *   route_weights_nvs R device pointers to rank q's [NvS] fp32, or NULL for
+ *                     the unweighted sum
+ *   out               [S,H] bf16 (16-byte aligned)
+ *   gathered_weights  [S,K] fp32 or NULL; = the weight of each slot read
+ */
+MOONEP_API int moonep_combine_rank(moonep_handle_t h, const moonep_plan_t *plan, const void *const *hidden_nvs,
+                                   const float *const *route_weights_nvs, void *out, float *gathered_weights,
+                                   moonep_stream_t stream);
+
+/*
  * moonep_plan without a handle and without allocating: the same plan as
  * moonep_plan for the same cfg and inputs.  (This entry point has no
  * counterpart on the pages; it exists for callers that cannot call cudaMalloc

@@ -27,7 +27,14 @@ struct moonep_handle {
     int grid_weights;
     void *ws_mem;
     Workspace ws;
+    Workspace ws_rank;  // one-rank planning (moonep_plan_rank): its own barrier counter and parity slots
 };
+
+// Handle workspace: [group planning][group GEMM pair table][one-rank planning]
+static size_t pair_table_offset(const Dims &d) { return (workspace_bytes(d) + 255) / 256 * 256; }
+static size_t rank_ws_offset(const Dims &d) {
+    return (pair_table_offset(d) + sizeof(int32_t) * (size_t)d.R * gemm_pair_slots(d) + 255) / 256 * 256;
+}
 
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -169,7 +176,7 @@ extern "C" int moonep_create(const moonep_config_t *cfg, moonep_handle_t *out) {
     h->grid_combine = h->sms * combine_blocks_per_sm(d.K);
     h->grid_weights = h->sms * weights_blocks_per_sm();
 
-    const size_t wsb = (workspace_bytes(d) + 255) / 256 * 256 + sizeof(int32_t) * (size_t)d.R * gemm_pair_slots(d);
+    const size_t wsb = rank_ws_offset(d) + workspace_bytes(d);
     if ((e = cudaMalloc(&h->ws_mem, wsb)) != cudaSuccess) { free(h); return fail_cuda(e); }
     if ((e = cudaMemset(h->ws_mem, 0, wsb)) != cudaSuccess) {
         cudaFree(h->ws_mem);
@@ -177,6 +184,7 @@ extern "C" int moonep_create(const moonep_config_t *cfg, moonep_handle_t *out) {
         return fail_cuda(e);
     }
     carve_workspace(d, h->ws_mem, &h->ws);
+    carve_workspace(d, static_cast<char *>(h->ws_mem) + rank_ws_offset(d), &h->ws_rank);
     *out = h;
     return MOONEP_OK;
 }
@@ -205,19 +213,56 @@ extern "C" int moonep_plan(moonep_handle_t h, const int32_t *topk, const int32_t
     a.d = h->d;
     a.topk = topk;
     a.tpe = tokens_per_expert;
+    a.src_rank = -1;
+    a.counts_all = nullptr;
     a.plan = *plan;
     a.ws = h->ws;
     const cudaError_t e = launch_plan(a, h->grid_plan, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? MOONEP_OK : fail_cuda(e);
 }
 
+extern "C" int moonep_plan_rank(moonep_handle_t h, int32_t rank, const int32_t *topk, const int32_t *counts_all,
+                                const moonep_plan_t *plan, moonep_stream_t stream) {
+    if (!h || !topk || !counts_all || !plan_ok(plan)) return MOONEP_ERR_NULL;
+    if (h->d.B > 0 && !plan->slot_expert) return MOONEP_ERR_NULL;
+    if (rank < 0 || rank >= h->d.R) return MOONEP_ERR_SIZE;
+    PlanArgs a;
+    a.d = h->d;
+    a.topk = topk;
+    a.tpe = nullptr;
+    a.src_rank = rank;
+    a.counts_all = counts_all;
+    a.plan = *plan;
+    a.ws = h->ws_rank;
+    const cudaError_t e = launch_plan(a, h->d.nch, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MOONEP_OK : fail_cuda(e);
+}
+
 static CopyArgs copy_args(moonep_handle_t h, const moonep_plan_t *plan) {
     CopyArgs a;
+    memset(&a, 0, sizeof(a));
     a.d = h->d;
     a.dst = plan->dst;
     a.status = plan->status;
     a.status_rw = plan->status;
+    a.ntok = (int64_t)h->d.R * h->d.S;
     return a;
+}
+
+// One rank's call: its own S tokens, the R ranks' buffers through tables.
+// Every buffer pointer is required and 16-byte aligned; the weight tables
+// are all given or all NULL.
+static int peer_tables(moonep_handle_t h, void *const *bufs, float *const *wbufs, CopyArgs *a) {
+    if (!bufs) return MOONEP_ERR_NULL;
+    a->ntok = h->d.S;
+    a->peered = 1;
+    for (int q = 0; q < h->d.R; ++q) {
+        if (!bufs[q] || (wbufs && !wbufs[q])) return MOONEP_ERR_NULL;
+        if (!aligned16(bufs[q])) return MOONEP_ERR_ALIGN;
+        a->peer[q] = bufs[q];
+        a->peer_w[q] = wbufs ? wbufs[q] : nullptr;
+    }
+    return MOONEP_OK;
 }
 
 extern "C" int moonep_dispatch(moonep_handle_t h, const moonep_plan_t *plan, const void *hidden,
@@ -233,6 +278,38 @@ extern "C" int moonep_dispatch(moonep_handle_t h, const moonep_plan_t *plan, con
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const cudaError_t e = h->bulk_dispatch ? launch_dispatch_bulk(a, h->grid_dispatch, st)
                                            : launch_dispatch(a, h->grid_dispatch, st);
+    return e == cudaSuccess ? MOONEP_OK : fail_cuda(e);
+}
+
+extern "C" int moonep_dispatch_rank(moonep_handle_t h, const moonep_plan_t *plan, const void *hidden,
+                                    const float *route_weights, void *const *hidden_nvs,
+                                    float *const *route_weights_nvs, moonep_stream_t stream) {
+    if (!h || !plan || !plan->dst || !plan->status || !hidden) return MOONEP_ERR_NULL;
+    if (!aligned16(hidden)) return MOONEP_ERR_ALIGN;
+    CopyArgs a = copy_args(h, plan);
+    const int rc = peer_tables(h, hidden_nvs, route_weights_nvs, &a);
+    if (rc != MOONEP_OK) return rc;
+    a.src = hidden;
+    a.w = route_weights;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const cudaError_t e = h->bulk_dispatch ? launch_dispatch_bulk(a, h->grid_dispatch, st)
+                                           : launch_dispatch(a, h->grid_dispatch, st);
+    return e == cudaSuccess ? MOONEP_OK : fail_cuda(e);
+}
+
+extern "C" int moonep_combine_rank(moonep_handle_t h, const moonep_plan_t *plan, const void *const *hidden_nvs,
+                                   const float *const *route_weights_nvs, void *out, float *gathered_weights,
+                                   moonep_stream_t stream) {
+    if (!h || !plan || !plan->dst || !plan->status || !out) return MOONEP_ERR_NULL;
+    if (!aligned16(out)) return MOONEP_ERR_ALIGN;
+    CopyArgs a = copy_args(h, plan);
+    // the kernel only reads through these tables
+    const int rc = peer_tables(h, const_cast<void *const *>(hidden_nvs),
+                               const_cast<float *const *>(route_weights_nvs), &a);
+    if (rc != MOONEP_OK) return rc;
+    a.out = out;
+    a.w_out = route_weights_nvs ? gathered_weights : nullptr;
+    const cudaError_t e = launch_combine(a, h->grid_combine, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? MOONEP_OK : fail_cuda(e);
 }
 
@@ -303,7 +380,7 @@ extern "C" int moonep_group_gemm(moonep_handle_t h, const moonep_plan_t *plan, c
         return MOONEP_ERR_ALIGN;
     const int rc = gemm_supported(h->d, Hp);
     if (rc != MOONEP_OK) return rc;
-    int32_t *pairs = reinterpret_cast<int32_t *>(static_cast<char *>(h->ws_mem) + (workspace_bytes(h->d) + 255) / 256 * 256);
+    int32_t *pairs = reinterpret_cast<int32_t *>(static_cast<char *>(h->ws_mem) + pair_table_offset(h->d));
     return launch_group_gemm(h->d, plan, x_nvs, weights, pool, y_nvs, Hp, pairs, reinterpret_cast<cudaStream_t>(stream));
 }
 

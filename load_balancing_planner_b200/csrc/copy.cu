@@ -15,41 +15,58 @@ namespace moonep {
 __device__ __forceinline__ uint4 ld_stream(const uint4 *p) { return __ldcs(p); }
 __device__ __forceinline__ void st_stream(uint4 *p, const uint4 &v) { __stcs(p, v); }
 
+// Slot dk = q*NvS + i of the group: row dk of the one buffer `base`, or row i
+// of rank q's own buffer when the call is peered.  `row` is in units of T.
+template <typename T>
+__device__ __forceinline__ T *slot_row(const CopyArgs &a, T *base, int dk, int64_t row) {
+    if (!a.peered) return base + (int64_t)dk * row;
+    const int q = dk / a.d.nvs;
+    return static_cast<T *>(a.peer[q]) + (int64_t)(dk - q * a.d.nvs) * row;
+}
+// the route weight of slot dk, or NULL when the call carries none
+__device__ __forceinline__ float *slot_weight(const CopyArgs &a, float *base, int dk) {
+    if (!a.peered) return base ? base + dk : nullptr;
+    const int q = dk / a.d.nvs;
+    return a.peer_w[q] ? a.peer_w[q] + (dk - q * a.d.nvs) : nullptr;
+}
+template <typename T>
+__device__ __forceinline__ T *shfl_ptr(T *p, int src) {
+    return reinterpret_cast<T *>(__shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(p), src));
+}
+
 // ---- dispatch ----------------------------------------------------------------
 // KT > 0: K known at compile time, the K destination rows are broadcast into
 // registers once per token; KT == 0: any K, one shuffle per row and step.
 template <int KT, int U>
-__global__ void __launch_bounds__(256) dispatch_kernel(CopyArgs a) {
+__global__ void __launch_bounds__(256) dispatch_kernel(const __grid_constant__ CopyArgs a) {
     pdl_wait();
     if (*a.status != 0) return;
     const Dims &d = a.d;
     const int K = KT > 0 ? KT : d.K;
     const int lane = threadIdx.x & 31;
     const int HV = d.H >> 3;
-    const int64_t ntok = (int64_t)d.R * d.S;
+    const int64_t ntok = a.ntok;
     const int64_t nslots = (int64_t)d.R * d.nvs;
     const uint4 *src = static_cast<const uint4 *>(a.src);
     uint4 *buf = static_cast<uint4 *>(a.out);
     const int64_t wstride = ((int64_t)gridDim.x * blockDim.x) >> 5;
     for (int64_t tok = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; tok < ntok; tok += wstride) {
-        int dk = -1;
+        uint4 *mine = nullptr;  // lane k: the row of the token's k-th slot
         if (lane < K) {
-            dk = a.dst[tok * K + lane];
+            const int dk = a.dst[tok * K + lane];
             if (dk < 0 || dk >= nslots) {
                 atomicOr(a.status_rw, MOONEP_STATUS_BAD_PLAN);
-                dk = -1;
-            } else if (a.w != nullptr && a.w_out != nullptr) {
-                a.w_out[dk] = __ldcs(a.w + tok * K + lane);
+            } else {
+                mine = slot_row(a, buf, dk, HV);
+                float *wo = slot_weight(a, a.w_out, dk);
+                if (a.w != nullptr && wo != nullptr) *wo = __ldcs(a.w + tok * K + lane);
             }
         }
         const uint4 *row = src + tok * HV;
         if constexpr (KT > 0) {
             uint4 *orow[KT];
 #pragma unroll
-            for (int k = 0; k < KT; ++k) {
-                const int dd = __shfl_sync(0xffffffffu, dk, k);
-                orow[k] = dd < 0 ? nullptr : buf + (int64_t)dd * HV;
-            }
+            for (int k = 0; k < KT; ++k) orow[k] = shfl_ptr(mine, k);
             for (int v0 = 0; v0 < HV; v0 += 32 * U) {
                 uint4 x[U];
 #pragma unroll
@@ -76,9 +93,8 @@ __global__ void __launch_bounds__(256) dispatch_kernel(CopyArgs a) {
                     if (v < HV) x[u] = ld_stream(row + v);
                 }
                 for (int k = 0; k < K; ++k) {
-                    const int dd = __shfl_sync(0xffffffffu, dk, k);
-                    if (dd < 0) continue;
-                    uint4 *o = buf + (int64_t)dd * HV;
+                    uint4 *o = shfl_ptr(mine, k);
+                    if (o == nullptr) continue;
 #pragma unroll
                     for (int u = 0; u < U; ++u) {
                         const int v = v0 + u * 32 + lane;
@@ -102,7 +118,7 @@ constexpr int kBulkMinRow = 2048;
 constexpr int kBulkStages = 3;
 // one warp per block; NS stages of `rowbytes` each, then NS mbarriers
 template <int KT>
-__global__ void __launch_bounds__(32) dispatch_bulk_kernel(CopyArgs a) {
+__global__ void __launch_bounds__(32) dispatch_bulk_kernel(const __grid_constant__ CopyArgs a) {
     extern __shared__ __align__(128) uint8_t sm[];
     pdl_wait();
     if (*a.status != 0) return;
@@ -110,7 +126,7 @@ __global__ void __launch_bounds__(32) dispatch_bulk_kernel(CopyArgs a) {
     const int K = KT > 0 ? KT : d.K;
     const int lane = threadIdx.x;
     const uint32_t rowbytes = (uint32_t)d.H * 2u;
-    const int64_t ntok = (int64_t)d.R * d.S;
+    const int64_t ntok = a.ntok;
     const int64_t nslots = (int64_t)d.R * d.nvs;
     const uint8_t *src = static_cast<const uint8_t *>(a.src);
     uint8_t *buf = static_cast<uint8_t *>(a.out);
@@ -134,22 +150,23 @@ __global__ void __launch_bounds__(32) dispatch_bulk_kernel(CopyArgs a) {
         const int64_t tok = tok_of(i);
         const int s = (int)(i % kBulkStages);
         const uint32_t parity = (uint32_t)((i / kBulkStages) & 1);
-        int dk = -1;
+        uint8_t *mine = nullptr;  // lane k: the row of the token's k-th slot
         if (lane < K) {
-            dk = a.dst[tok * K + lane];
+            const int dk = a.dst[tok * K + lane];
             if (dk < 0 || dk >= nslots) {
                 atomicOr(a.status_rw, MOONEP_STATUS_BAD_PLAN);
-                dk = -1;
-            } else if (a.w != nullptr && a.w_out != nullptr) {
-                a.w_out[dk] = __ldcs(a.w + tok * K + lane);
+            } else {
+                mine = slot_row(a, buf, dk, rowbytes);
+                float *wo = slot_weight(a, a.w_out, dk);
+                if (a.w != nullptr && wo != nullptr) *wo = __ldcs(a.w + tok * K + lane);
             }
         }
         if (lane == 0) ok = mbar_wait(bar0 + 8u * s, parity);
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         if (!ok) break;
         for (int k = 0; k < K; ++k) {
-            const int dd = __shfl_sync(0xffffffffu, dk, k);
-            if (lane == 0 && dd >= 0) bulk_store(buf + (int64_t)dd * rowbytes, stage0 + s * rowbytes, rowbytes, pol);
+            uint8_t *o = shfl_ptr(mine, k);
+            if (lane == 0 && o != nullptr) bulk_store(o, stage0 + s * rowbytes, rowbytes, pol);
         }
         if (lane == 0) {
             bulk_commit();
@@ -201,30 +218,34 @@ __device__ __forceinline__ uint4 pack_bf16x8(const float (&acc)[8]) {
 // KT > 0: K known at compile time (all K*U loads of a step in flight);
 // KT == 0: any K, loads issued in groups of 4 rows.
 template <int KT, int U>
-__global__ void __launch_bounds__(256) combine_kernel(CopyArgs a) {
+__global__ void __launch_bounds__(256) combine_kernel(const __grid_constant__ CopyArgs a) {
     pdl_wait();
     if (*a.status != 0) return;
     const Dims &d = a.d;
     const int K = KT > 0 ? KT : d.K;
     const int lane = threadIdx.x & 31;
     const int HV = d.H >> 3;
-    const int64_t ntok = (int64_t)d.R * d.S;
+    const int64_t ntok = a.ntok;
     const int64_t nslots = (int64_t)d.R * d.nvs;
-    const uint4 *y = static_cast<const uint4 *>(a.src);
+    const uint4 *y = static_cast<const uint4 *>(a.peered ? a.peer[0] : a.src);
+    // weighted: route_weights_nvs given (one buffer, or every rank's when peered)
+    const bool weighted = a.peered ? a.peer_w[0] != nullptr : a.w != nullptr;
     uint4 *out = static_cast<uint4 *>(a.out);
     const int64_t wstride = ((int64_t)gridDim.x * blockDim.x) >> 5;
     for (int64_t tok = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; tok < ntok; tok += wstride) {
-        int dk = 0;
+        const uint4 *mine = y;  // lane k: the row of the token's k-th slot (a valid row on every lane)
         float wk = 1.0f;
         if (lane < K) {
-            dk = a.dst[tok * K + lane];
+            const int dk = a.dst[tok * K + lane];
             if (dk < 0 || dk >= nslots) {
                 atomicOr(a.status_rw, MOONEP_STATUS_BAD_PLAN);
-                dk = 0;
                 wk = 0.0f;
-            } else if (a.w != nullptr) {
-                wk = a.w[dk];
-                if (a.w_out != nullptr) a.w_out[tok * K + lane] = wk;
+            } else {
+                mine = slot_row(a, y, dk, HV);
+                if (weighted) {
+                    wk = *slot_weight(a, const_cast<float *>(a.w), dk);
+                    if (a.w_out != nullptr) a.w_out[tok * K + lane] = wk;
+                }
             }
         }
         uint4 *orow = out + tok * HV;
@@ -238,8 +259,7 @@ __global__ void __launch_bounds__(256) combine_kernel(CopyArgs a) {
                 uint4 yv[KT][U];
 #pragma unroll
                 for (int k = 0; k < KT; ++k) {
-                    const int dd = __shfl_sync(0xffffffffu, dk, k);
-                    const uint4 *yrow = y + (int64_t)dd * HV;
+                    const uint4 *yrow = shfl_ptr(mine, k);
 #pragma unroll
                     for (int u = 0; u < U; ++u) {
                         const int v = v0 + u * 32 + lane;
@@ -257,8 +277,7 @@ __global__ void __launch_bounds__(256) combine_kernel(CopyArgs a) {
                     uint4 yv[4][U];
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
-                        const int dd = __shfl_sync(0xffffffffu, dk, (k0 + kk) & 31);
-                        const uint4 *yrow = y + (int64_t)dd * HV;
+                        const uint4 *yrow = shfl_ptr(mine, (k0 + kk) & 31);
 #pragma unroll
                         for (int u = 0; u < U; ++u) {
                             const int v = v0 + u * 32 + lane;

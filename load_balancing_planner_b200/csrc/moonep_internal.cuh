@@ -41,8 +41,10 @@ void carve_workspace(const Dims &d, void *base, Workspace *ws);
 
 struct PlanArgs {
     Dims d;
-    const int32_t *topk;
-    const int32_t *tpe;
+    const int32_t *topk;        // [R,S,K], or [S,K] of src_rank
+    const int32_t *tpe;         // [R,E] router counts to check, or NULL (group planning)
+    int src_rank;               // -1: plan the whole group; else this rank's picks only
+    const int32_t *counts_all;  // [R,E] every rank's counts (src_rank >= 0)
     moonep_plan_t plan;
     Workspace ws;
 };
@@ -58,10 +60,17 @@ struct CopyArgs {
     const int32_t *dst;
     const int32_t *status;
     int32_t *status_rw;
-    const void *src;  // dispatch: hidden [R,S,H]; combine: y [R,NvS,H]
-    const float *w;   // dispatch: route_weights [R,S,K]; combine: route_weights_nvs
-    void *out;        // dispatch: hidden_nvs; combine: out [R,S,H]
-    float *w_out;     // dispatch: route_weights_nvs; combine: gathered weights [R,S,K]
+    int64_t ntok;     // token rows: R*S (the group), S (one rank)
+    const void *src;  // dispatch: hidden [ntok,H]; combine: y [R,NvS,H] (unless peered)
+    const float *w;   // dispatch: route_weights [ntok,K]; combine: route_weights_nvs (unless peered)
+    void *out;        // dispatch: hidden_nvs (unless peered); combine: out [ntok,H]
+    float *w_out;     // dispatch: route_weights_nvs (unless peered); combine: gathered weights [ntok,K]
+    // peered: slot dst = q*NvS + i lives at row i of rank q's own buffer
+    // peer[q] (dispatch writes it, combine reads it), its route weight at
+    // peer_w[q][i] (all NULL: no weights)
+    int peered;
+    void *peer[MOONEP_MAX_R];
+    float *peer_w[MOONEP_MAX_R];
 };
 
 cudaError_t launch_dispatch(const CopyArgs &a, int grid, cudaStream_t st);

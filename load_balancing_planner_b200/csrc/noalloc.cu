@@ -60,6 +60,8 @@ extern "C" int moonep_plan_noalloc(const moonep_config_t *cfg, const int32_t *to
     a.d = d;
     a.topk = topk;
     a.tpe = tokens_per_expert;
+    a.src_rank = -1;
+    a.counts_all = nullptr;
     a.plan = *plan;
     carve_workspace(d, base, &a.ws);
     // The array keeps the previous call's contents.  What must start at zero

@@ -302,7 +302,10 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
     uint16_t *ent_rank = reinterpret_cast<uint16_t *>(reinterpret_cast<uint8_t *>(ent_e) +
                                                       align256(sizeof(uint16_t) * (size_t)d.ct * K));
     int32_t *tpe_s = reinterpret_cast<int32_t *>(smem + region1_bytes(d) + ent_bytes(d));  // [R][E], block 0
-    const bool checker = blockIdx.x == 0 && a.tpe != nullptr;
+    // one_rank: the grid covers one source rank's chunks, and the per-rank
+    // counts come from the caller (every rank's router counts, gathered)
+    const bool one_rank = a.src_rank >= 0;
+    const bool checker = blockIdx.x == 0 && (one_rank || a.tpe != nullptr);
     const int CW = d.cw;
     uint16_t *wcnt = reinterpret_cast<uint16_t *>(region1);                       // [CW][E]
     uint32_t *wmask = reinterpret_cast<uint32_t *>(region1 + counts_bytes(d));    // [CW][E]
@@ -313,7 +316,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
     // the plan's status starts at 0 (block 0, before the grid barrier); every
     // later update is an atomicOr, so no error bit can be overwritten
     if (blockIdx.x == 0 && tid == 0) *a.plan.status = 0;
-    if (checker && tpe_in_smem(d))
+    if (checker && !one_rank && tpe_in_smem(d))
         for (int i = tid; i < R * E; i += kPlanThreads) tpe_s[i] = __ldg(a.tpe + i);
 
     __shared__ unsigned long long s_call;
@@ -324,12 +327,13 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
     }
 
     PLAN_TRACE(0);
-    const int row = blockIdx.x;  // histogram row = r * nch + c
+    const int row = one_rank ? a.src_rank * d.nch + (int)blockIdx.x : (int)blockIdx.x;  // histogram row = r * nch + c
     const int r = row / d.nch, c = row - r * d.nch;
     const int t0 = c * d.ct;
     const int t1 = min(d.S, t0 + d.ct);
     const int n_ent = (t1 - t0) * K;
-    const int64_t base = ((int64_t)r * d.S + t0) * K;
+    // picks (and their dst) of this chunk: [R,S,K] for the group, [S,K] for one rank
+    const int64_t base = ((one_rank ? 0 : (int64_t)r * d.S) + t0) * K;
 
     // ---------------- A. count ----------------
     int bad = 0;
@@ -475,7 +479,8 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
     // compiler keeps them all in flight.)
     bool mismatch = false;
     {
-        const int32_t *cnt = a.ws.cnt + (size_t)parity * R * E;
+        const int32_t *cnt = one_rank ? a.counts_all : a.ws.cnt + (size_t)parity * R * E;
+        const int32_t *own = a.ws.cnt + ((size_t)parity * R + r) * E;  // this call's picks of rank r
         const int32_t *mine_rows = a.ws.hist + (int64_t)r * d.nch * E;
         // rows q < R are the per-rank counts, rows R <= q < R + c this rank's
         // earlier chunk histograms; 16 loads in flight per batch
@@ -497,7 +502,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
                         tot += v[u];
                         if (q < r) mypre += v[u];
                         if (q == r) myv = v[u];
-                        if (checker) {
+                        if (checker && !one_rank) {
                             const int t = tpe_in_smem(d) ? tpe_s[q * E + e] : __ldg(a.tpe + (int64_t)q * E + e);
                             if (t != v[u]) mismatch = true;
                         }
@@ -508,7 +513,8 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
             }
             T[e] = tot;
             pre[e] = mypre;
-            if (c == 0) a.plan.counts[(int64_t)r * E + e] = myv;
+            if (c == 0 && !one_rank) a.plan.counts[(int64_t)r * E + e] = myv;
+            if (checker && one_rank && ld_cg(own + e) != myv) mismatch = true;  // the rank's own row
         }
     }
     // the router's counts are checked by block 0 only, which writes the
@@ -516,8 +522,38 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
     __shared__ int s_mismatch;
     if (tid == 0) s_mismatch = 0;
     const int mm = __reduce_or_sync(0xffffffffu, mismatch ? 1 : 0);
+    __shared__ int s_cbad;
+    if (tid == 0) s_cbad = 0;
     __syncthreads();
     if (lane == 0 && mm) atomicOr(&s_mismatch, MOONEP_STATUS_COUNT_MISMATCH);
+    // One rank: the gathered counts must hold S*K non-negative picks per rank,
+    // or the layout below is undefined.  Every block checks every row, so all
+    // take the same decision; block 0 copies the rows into the plan.
+    if (one_rank) {
+        for (int q = w; q < R; q += kPlanWarps) {
+            const int32_t *row = a.counts_all + (int64_t)q * E;
+            long long sum = 0;
+            bool neg = false;
+            for (int e0 = 0; e0 < E; e0 += 32 * 8) {
+                int v[8];  // all loads of a batch in flight before any store
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int e = e0 + 32 * u + lane;
+                    v[u] = e < E ? ld_cg(row + e) : 0;
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int e = e0 + 32 * u + lane;
+                    neg |= v[u] < 0;
+                    sum += v[u];
+                    if (blockIdx.x == 0 && e < E) a.plan.counts[(int64_t)q * E + e] = v[u];
+                }
+            }
+            for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+            const bool rowbad = __any_sync(0xffffffffu, neg) || sum != (long long)d.S * K;
+            if (lane == 0 && rowbad) atomicOr(&s_cbad, MOONEP_STATUS_COUNT_MISMATCH);
+        }
+    }
     // group loads and the largest count
     int mx = 0;
     for (int e = tid; e < E; e += kPlanThreads) mx = max(mx, T[e]);
@@ -531,8 +567,8 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
     }
     __syncthreads();
     PLAN_TRACE(2);
-    if (s_status != 0) {
-        if (blockIdx.x == 0 && tid == 0) atomicOr(a.plan.status, s_status | s_mismatch);
+    if (s_status != 0 || s_cbad != 0) {
+        if (blockIdx.x == 0 && tid == 0) atomicOr(a.plan.status, s_status | s_mismatch | s_cbad);
         return;
     }
 

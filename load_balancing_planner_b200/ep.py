@@ -1,0 +1,96 @@
+"""One rank of a real expert-parallel group: the per-rank form of `Buffer`.
+
+On R GPUs each rank holds only its own router output (MoonEP README,
+"dispatch fwd": `tokens_per_expert` is the rank's local count), and the
+dispatched buffers of the R ranks live on R devices.  The planner needs, besides
+the rank's picks, every rank's counts: one all-gather of R x E int32
+(`gather_counts`), after which every rank derives the same layout and writes
+the slots of its own picks (`moonep_plan_rank`).  Dispatch and combine address
+the R ranks' buffers through a table of their device pointers
+(`moonep_dispatch_rank`, `moonep_combine_rank`).
+
+`RankBuffer` takes those buffers as a list of R tensors.  On a real group
+they are this rank's views of the peers' memory (peer-mapped allocations,
+e.g. from torch's symmetric memory); on one GPU they are R separate local
+allocations, which is how the tests run it.  Argument marshalling only: every
+step runs in the library's kernels, and the gather is a torch.distributed
+collective of the caller's process group.
+"""
+from __future__ import annotations
+
+import torch
+import torch.distributed as dist
+
+from . import moonep
+
+
+def gather_counts(tokens_per_expert: torch.Tensor, group=None) -> torch.Tensor:
+    """[R, E] int32: row q = rank q's tokens_per_expert [E], in group rank
+    order, identical on every rank (one all-gather)."""
+    if tokens_per_expert.dim() != 1 or tokens_per_expert.dtype != torch.int32:
+        raise ValueError("tokens_per_expert: expected an [E] int32 tensor")
+    world = dist.get_world_size(group)
+    rows = [torch.empty_like(tokens_per_expert) for _ in range(world)]
+    dist.all_gather(rows, tokens_per_expert.contiguous(), group=group)
+    return torch.stack(rows)
+
+
+class RankBuffer:
+    """Rank `rank` of an EP group of `num_ep_ranks`: S tokens, hidden size H,
+    top-K over E experts, B prefetch slots.
+
+    `hidden_nvs`: the R ranks' dispatched buffers, a list of R [NvS, H] bf16
+    tensors (entry `rank` is this rank's own); `route_weights_nvs` the same
+    for the [NvS] fp32 weights, or None.  NvS is `self.nvs`, known before any
+    buffer exists (`RankBuffer.nvs_of`)."""
+
+    def __init__(self, S: int, H: int, K: int, E: int, num_ep_ranks: int, rank: int, hidden_nvs,
+                 route_weights_nvs=None, token_padding: int = 128, B: int | None = None,
+                 mode: int = moonep.TRAINING, num_sms: int | None = None):
+        if not 0 <= rank < num_ep_ranks:
+            raise ValueError(f"rank {rank} outside [0, {num_ep_ranks})")
+        self.handle = moonep.moonep_create(S, H, K, E, num_ep_ranks, B, token_padding, num_sms or 0, mode)
+        self.rank, self.R = rank, num_ep_ranks
+        self.S, self.H, self.K, self.E, self.B = S, H, K, E, self.handle.B
+        self.nvs = self.handle.nvs
+        self.hidden_nvs = list(hidden_nvs)
+        self.route_weights_nvs = None if route_weights_nvs is None else list(route_weights_nvs)
+
+    @staticmethod
+    def nvs_of(S: int, K: int, E: int, num_ep_ranks: int, token_padding: int = 128) -> int:
+        """Slots of one rank's buffer, as moonep_nvs computes them."""
+        G, tp = E // num_ep_ranks, token_padding
+        n = S * K + 2 * G * (tp - 1)
+        return (n + tp - 1) // tp * tp
+
+    def plan(self, topk, tokens_per_expert=None, *, counts_all=None, group=None) -> moonep.Plan:
+        """This rank's plan from its picks topk [S,K] and the gathered counts:
+        `counts_all` [R,E] when the caller has it, else gathered here from
+        `tokens_per_expert` [E] over `group`."""
+        if counts_all is None:
+            if tokens_per_expert is None:
+                raise ValueError("plan needs tokens_per_expert or counts_all")
+            counts_all = gather_counts(tokens_per_expert, group)
+        return moonep.moonep_plan_rank(self.handle, self.rank, topk, counts_all)
+
+    def dispatch(self, plan: moonep.Plan, hidden, route_weights=None):
+        """Scatter this rank's rows hidden [S,H] (route_weights [S,K]) into
+        the R ranks' buffers.  The receivers may read their buffer once every
+        rank's dispatch has completed (a barrier of the caller's group)."""
+        w_nvs = self.route_weights_nvs if route_weights is not None else None
+        moonep.moonep_dispatch_rank(self.handle, plan, hidden, route_weights, self.hidden_nvs, w_nvs)
+
+    def combine(self, plan: moonep.Plan, expert_out_nvs, weighted: bool = True, out=None):
+        """out [S,H] = bf16(sum_k w_k * y[slot of (t,k)]) over this rank's
+        tokens, reading `expert_out_nvs` (the R ranks' [NvS,H] outputs, a list
+        like hidden_nvs) and, when weighted, the route weights that dispatch
+        placed.  Returns (out, gathered_weights [S,K] or None)."""
+        w_nvs = self.route_weights_nvs if weighted else None
+        if weighted and w_nvs is None:
+            raise ValueError("weighted combine needs route_weights_nvs")
+        return moonep.moonep_combine_rank(self.handle, plan, list(expert_out_nvs), w_nvs, out)
+
+    def destroy(self) -> None:
+        if self.handle is not None:
+            self.handle.close()
+            self.handle = None

@@ -60,6 +60,9 @@ def _load():
         "moonep_last_error": ([], ctypes.c_char_p),
         "moonep_plan_noalloc": ([ctypes.POINTER(Config), P, P, ctypes.POINTER(PlanStruct), P], ctypes.c_int),
         "moonep_group_gemm": ([P, ctypes.POINTER(PlanStruct), P, P, P, P, i64, P], ctypes.c_int),
+        "moonep_plan_rank": ([P, i32, P, P, ctypes.POINTER(PlanStruct), P], ctypes.c_int),
+        "moonep_dispatch_rank": ([P, ctypes.POINTER(PlanStruct), P, P, P, P, P], ctypes.c_int),
+        "moonep_combine_rank": ([P, ctypes.POINTER(PlanStruct), P, P, P, P, P], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -72,7 +75,7 @@ lib = _load()
 EXPORTS = ("moonep_create", "moonep_destroy", "moonep_nvs", "moonep_get_config", "moonep_plan",
            "moonep_dispatch", "moonep_combine", "moonep_prefetch_weight", "moonep_reduce_grad",
            "moonep_read_status", "moonep_error_string", "moonep_last_error", "moonep_plan_noalloc",
-           "moonep_group_gemm")
+           "moonep_group_gemm", "moonep_plan_rank", "moonep_dispatch_rank", "moonep_combine_rank")
 NOALLOC_SCRATCH_BYTES = 1 << 20
 
 
@@ -134,13 +137,15 @@ class Handle:
 
 class Plan:
     """Device arrays of one plan (caller-owned, see moonep_plan_t).  `h` is a
-    Handle, or a Config for moonep_plan_noalloc."""
+    Handle, or a Config for moonep_plan_noalloc.  `rank` marks one rank's
+    plan (moonep_plan_rank): dst is then [S,K]."""
 
-    def __init__(self, h, device=None):
+    def __init__(self, h, device=None, rank: int | None = None):
         dev = device or torch.device("cuda", torch.cuda.current_device())
         R, S, K, E, B = h.R, h.S, h.K, h.E, h.B
         i32 = dict(dtype=torch.int32, device=dev)
-        self.dst = torch.empty((R, S, K), **i32)
+        self.rank = rank
+        self.dst = torch.empty((S, K) if rank is not None else (R, S, K), **i32)
         self.cu_seqlens = torch.empty((R, E + B), **i32)
         self.row_counts = torch.empty((R, E + B), **i32)
         self.slot_expert = torch.empty((R, max(B, 1)), **i32)
@@ -194,8 +199,73 @@ def moonep_plan_noalloc(cfg: Config, topk, tokens_per_expert=None, plan: Plan | 
     return plan
 
 
+def _group_plan(plan: Plan, what: str):
+    if plan.rank is not None:
+        raise ValueError(f"{what} takes a group plan; use the _rank call with a rank's plan")
+
+
+def _rank_plan(plan: Plan, what: str):
+    if plan.rank is None:
+        raise ValueError(f"{what} takes a plan from moonep_plan_rank")
+
+
+def moonep_plan_rank(h: Handle, rank: int, topk, counts_all, plan: Plan | None = None, stream=None) -> Plan:
+    """One rank's plan from its own picks topk [S,K] and every rank's router
+    counts counts_all [R,E] (row q = rank q's tokens_per_expert)."""
+    _expect(topk, (h.S, h.K), torch.int32, "topk")
+    _expect(counts_all, (h.R, h.E), torch.int32, "counts_all")
+    plan = plan or Plan(h, topk.device, rank=rank)
+    _rank_plan(plan, "moonep_plan_rank")
+    plan.rank = rank
+    _check(lib.moonep_plan_rank(h.ptr, rank, _ptr(topk), _ptr(counts_all), ctypes.byref(plan.struct),
+                                _stream(stream)), "moonep_plan_rank")
+    return plan
+
+
+def moonep_dispatch_rank(h: Handle, plan: Plan, hidden, route_weights, hidden_nvs, route_weights_nvs=None,
+                         stream=None):
+    """Scatter one rank's rows hidden [S,H] (and route_weights [S,K]) into the
+    R ranks' buffers: hidden_nvs is a list of R [NvS,H] bf16 tensors,
+    route_weights_nvs None or a list of R [NvS] fp32 tensors."""
+    _rank_plan(plan, "moonep_dispatch_rank")
+    _expect(hidden, (h.S, h.H), torch.bfloat16, "hidden")
+    _expect(route_weights, (h.S, h.K), torch.float32, "route_weights")
+    bufs, wbufs = _rank_tables(h, hidden_nvs, route_weights_nvs)
+    _check(lib.moonep_dispatch_rank(h.ptr, ctypes.byref(plan.struct), _ptr(hidden), _ptr(route_weights),
+                                    bufs, wbufs, _stream(stream)), "moonep_dispatch_rank")
+
+
+def moonep_combine_rank(h: Handle, plan: Plan, hidden_nvs, route_weights_nvs=None, out=None,
+                        gathered_weights=None, gather=True, stream=None):
+    """out [S,H] = the weighted sum of each own token's K slots, read from the
+    R ranks' buffers (lists as in moonep_dispatch_rank)."""
+    _rank_plan(plan, "moonep_combine_rank")
+    bufs, wbufs = _rank_tables(h, hidden_nvs, route_weights_nvs)
+    dev = hidden_nvs[0].device
+    if out is None:
+        out = torch.empty((h.S, h.H), dtype=torch.bfloat16, device=dev)
+    if gather and route_weights_nvs is not None and gathered_weights is None:
+        gathered_weights = torch.empty((h.S, h.K), dtype=torch.float32, device=dev)
+    _expect(out, (h.S, h.H), torch.bfloat16, "out")
+    _expect(gathered_weights, (h.S, h.K), torch.float32, "gathered_weights")
+    _check(lib.moonep_combine_rank(h.ptr, ctypes.byref(plan.struct), bufs, wbufs, _ptr(out),
+                                   _ptr(gathered_weights), _stream(stream)), "moonep_combine_rank")
+    return out, gathered_weights
+
+
+def _rank_tables(h: Handle, hidden_nvs, route_weights_nvs):
+    if len(hidden_nvs) != h.R or (route_weights_nvs is not None and len(route_weights_nvs) != h.R):
+        raise ValueError("one buffer per rank")
+    for b in hidden_nvs:
+        _expect(b, (h.nvs, h.H), torch.bfloat16, "hidden_nvs[q]")
+    for b in route_weights_nvs or ():
+        _expect(b, (h.nvs,), torch.float32, "route_weights_nvs[q]")
+    return _ptr_array(hidden_nvs), (_ptr_array(route_weights_nvs) if route_weights_nvs is not None else None)
+
+
 def moonep_dispatch(h: Handle, plan: Plan, hidden, route_weights=None, hidden_nvs=None,
                     route_weights_nvs=None, stream=None):
+    _group_plan(plan, "moonep_dispatch")
     _expect(hidden, (h.R, h.S, h.H), torch.bfloat16, "hidden")
     _expect(route_weights, (h.R, h.S, h.K), torch.float32, "route_weights")
     if hidden_nvs is None:
@@ -211,6 +281,7 @@ def moonep_dispatch(h: Handle, plan: Plan, hidden, route_weights=None, hidden_nv
 
 def moonep_combine(h: Handle, plan: Plan, hidden_nvs, route_weights_nvs=None, out=None,
                    gathered_weights=None, gather=True, stream=None):
+    _group_plan(plan, "moonep_combine")
     _expect(hidden_nvs, (h.R, h.nvs, h.H), torch.bfloat16, "hidden_nvs")
     _expect(route_weights_nvs, (h.R, h.nvs), torch.float32, "route_weights_nvs")
     if out is None:

@@ -75,6 +75,9 @@ def test_null_arguments_are_rejected():
     assert moonep.lib.moonep_combine(None, None, None, None, None, None, None) == moonep.ERR_NULL
     assert moonep.lib.moonep_prefetch_weight(None, None, 1, None, None, 8, None) == moonep.ERR_NULL
     assert moonep.lib.moonep_reduce_grad(None, None, 1, None, None, 8, None) == moonep.ERR_NULL
+    assert moonep.lib.moonep_plan_rank(None, 0, None, None, None, None) == moonep.ERR_NULL
+    assert moonep.lib.moonep_dispatch_rank(None, None, None, None, None, None, None) == moonep.ERR_NULL
+    assert moonep.lib.moonep_combine_rank(None, None, None, None, None, None, None) == moonep.ERR_NULL
     assert moonep.lib.moonep_destroy(None) == moonep.OK
     assert moonep.lib.moonep_nvs(None) < 0
 

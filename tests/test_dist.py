@@ -62,3 +62,43 @@ def test_aggregate_value_counts_all_ranks():
     import bench
     assert bench.aggregate_gbs(1e9, 10, 4, 1000.0) == pytest.approx(40.0)
     assert bench.rank_seed(3, 2) == 5
+
+
+def _gather_worker(rank, world, port, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import datetime
+    import torch
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    from load_balancing_planner_b200.ep import gather_counts
+    try:
+        # one EP group of `world` ranks: the same seeded routing everywhere,
+        # each rank keeping only its own picks and their local counts
+        tk, _, _ = synth.routing(world, 64, 4, 16, 1.5, "hot8", seed=7)
+        mine = torch.from_numpy(synth.local_counts(tk[rank:rank + 1], 16)[0].copy())
+        table = gather_counts(mine).numpy()
+        # what the rank planner needs: the group's counts in rank order, which
+        # the oracle accepts as the router counts of the group's picks
+        ok = np.array_equal(table, synth.local_counts(tk, 16))
+        st = oracle.plan(tk, 16, 8, 8, 0, table)["status"]
+        q.put((rank, bool(ok), int(st), table.tobytes()))
+    finally:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def test_two_rank_count_gather_gloo():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_gather_worker, args=(r, 2, port, q)) for r in range(2)]
+    for pr in procs:
+        pr.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for pr in procs:
+        pr.join(timeout=60)
+        assert pr.exitcode == 0
+    (_, ok0, st0, t0), (_, ok1, st1, t1) = res
+    assert ok0 and ok1
+    assert st0 == st1 == 0
+    assert t0 == t1, "every rank holds the same table"
