@@ -301,6 +301,39 @@ MOONEP_API int moonep_combine_rank(moonep_handle_t h, const moonep_plan_t *plan,
                                    moonep_stream_t stream);
 
 /*
+ * Weight prefetch of one rank (README "Weight buffer"): for each projection p
+ * and each used slot b of rank `rank`, pool[p][b] = the home copy of expert
+ * e = slot_expert[rank][b], read from its home rank q = e / G.
+ *   weights[p*R + q] [G,H,Hp] bf16  rank q's home experts of projection p
+ *                                   (peer mappings on a real group)
+ *   pool[p]          [B,H,Hp] bf16  this rank's prefetch slots
+ * The plan is this rank's (moonep_plan_rank) or the group's: only its
+ * slot_expert is read.  Same checks as moonep_prefetch_weight; ERR_SIZE when
+ * rank is outside [0, R).  Bit-identical to rank `rank`'s slots after
+ * moonep_prefetch_weight.
+ */
+MOONEP_API int moonep_prefetch_weight_rank(moonep_handle_t h, const moonep_plan_t *plan, int32_t rank, int32_t n_proj,
+                                           const void *const *weights, void *const *pool, int64_t Hp,
+                                           moonep_stream_t stream);
+
+/*
+ * Grad-slot reduction of one home rank (README "Grad buffer"): for each
+ * projection and each home expert e of rank `rank` held by at least one slot
+ * of any rank, grads[p][e - rank*G] += the slots holding e, in ascending
+ * (rank, slot) order in fp32; then those slots are set to +0.0.
+ *   grads[p]                 [G,H,Hp] fp32  this rank's home experts' gradients
+ *   reduce_buffers[p*R + q]  [B,H,Hp] fp32  rank q's slot gradients (peer
+ *                                           mappings on a real group); read,
+ *                                           and the consumed slots zeroed
+ * The R ranks' calls touch disjoint slots (each slot holds one expert, whose
+ * home is one rank).  Bit-identical to the home rank's share of
+ * moonep_reduce_grad.
+ */
+MOONEP_API int moonep_reduce_grad_rank(moonep_handle_t h, const moonep_plan_t *plan, int32_t rank, int32_t n_proj,
+                                       float *const *grads, float *const *reduce_buffers, int64_t Hp,
+                                       moonep_stream_t stream);
+
+/*
  * moonep_plan without a handle and without allocating: the same plan as
  * moonep_plan for the same cfg and inputs.  (This entry point has no
  * counterpart on the pages; it exists for callers that cannot call cudaMalloc

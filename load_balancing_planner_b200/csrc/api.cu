@@ -338,6 +338,7 @@ static int weight_args(moonep_handle_t h, const moonep_plan_t *plan, int32_t n_p
     a->status = plan->status;
     a->n_proj = n_proj;
     a->hhp = (int64_t)h->d.H * Hp;
+    a->rank = -1;
     for (int p = 0; p < n_proj; ++p) {
         if (!src[p] || !dst[p]) return MOONEP_ERR_NULL;
         if (!aligned16(src[p]) || !aligned16(dst[p])) return MOONEP_ERR_ALIGN;
@@ -365,6 +366,57 @@ extern "C" int moonep_reduce_grad(moonep_handle_t h, const moonep_plan_t *plan, 
     // the reduce buffers are the source (read, then zeroed), the grads the destination
     const int rc = weight_args(h, plan, n_proj, reinterpret_cast<const void *const *>(reduce_buffers),
                                reinterpret_cast<void *const *>(grads), Hp, &a);
+    if (rc != MOONEP_OK) return rc;
+    if (h->d.B == 0) return MOONEP_OK;
+    const cudaError_t e = launch_reduce_grad(a, h->grid_weights, h->sms, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MOONEP_OK : fail_cuda(e);
+}
+
+// One rank's weight call: its own tensors (own[p]) and every rank's tensor
+// of the other side (peers[p*R + q]).
+static int weight_args_rank(moonep_handle_t h, const moonep_plan_t *plan, int32_t rank, int32_t n_proj,
+                            void *const *own, const void *const *peers, int64_t Hp, WeightArgs *a) {
+    if (!h || !plan || !plan->status || !own || !peers) return MOONEP_ERR_NULL;
+    if (n_proj < 1 || n_proj > MOONEP_MAX_PROJ || Hp < 1 || rank < 0 || rank >= h->d.R) return MOONEP_ERR_SIZE;
+    if (h->d.B > 0 && !plan->slot_expert) return MOONEP_ERR_NULL;
+    memset(a, 0, sizeof(*a));
+    a->d = h->d;
+    a->slot_expert = plan->slot_expert;
+    a->status = plan->status;
+    a->n_proj = n_proj;
+    a->hhp = (int64_t)h->d.H * Hp;
+    a->rank = rank;
+    for (int p = 0; p < n_proj; ++p) {
+        if (!own[p]) return MOONEP_ERR_NULL;
+        if (!aligned16(own[p])) return MOONEP_ERR_ALIGN;
+        a->dst[p] = own[p];
+        for (int q = 0; q < h->d.R; ++q) {
+            const void *x = peers[(size_t)p * h->d.R + q];
+            if (!x) return MOONEP_ERR_NULL;
+            if (!aligned16(x)) return MOONEP_ERR_ALIGN;
+            a->peer[p][q] = x;
+        }
+    }
+    return MOONEP_OK;
+}
+
+extern "C" int moonep_prefetch_weight_rank(moonep_handle_t h, const moonep_plan_t *plan, int32_t rank, int32_t n_proj,
+                                           const void *const *weights, void *const *pool, int64_t Hp,
+                                           moonep_stream_t stream) {
+    WeightArgs a;
+    const int rc = weight_args_rank(h, plan, rank, n_proj, pool, weights, Hp, &a);
+    if (rc != MOONEP_OK) return rc;
+    if (h->d.B == 0) return MOONEP_OK;
+    const cudaError_t e = launch_prefetch(a, h->grid_weights, h->sms, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MOONEP_OK : fail_cuda(e);
+}
+
+extern "C" int moonep_reduce_grad_rank(moonep_handle_t h, const moonep_plan_t *plan, int32_t rank, int32_t n_proj,
+                                       float *const *grads, float *const *reduce_buffers, int64_t Hp,
+                                       moonep_stream_t stream) {
+    WeightArgs a;
+    const int rc = weight_args_rank(h, plan, rank, n_proj, reinterpret_cast<void *const *>(grads),
+                                    reinterpret_cast<const void *const *>(reduce_buffers), Hp, &a);
     if (rc != MOONEP_OK) return rc;
     if (h->d.B == 0) return MOONEP_OK;
     const cudaError_t e = launch_reduce_grad(a, h->grid_weights, h->sms, reinterpret_cast<cudaStream_t>(stream));

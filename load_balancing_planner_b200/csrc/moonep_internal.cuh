@@ -90,6 +90,13 @@ struct WeightArgs {
     int64_t hhp;                 // H * Hp elements per expert
     const void *src[MOONEP_MAX_PROJ];
     void *dst[MOONEP_MAX_PROJ];
+    // rank < 0: the group (src/dst span all experts [E,..] and all slots
+    // [R*B,..]).  rank >= 0: that rank's share.  Its own side is dst (prefetch:
+    // its slots [B,..]) or dst (reduce_grad: its home experts [G,..]); the
+    // other side is every rank's tensor, peer[p][q] = rank q's home experts
+    // [G,..] (prefetch) or slots [B,..] (reduce_grad).
+    int rank;
+    const void *peer[MOONEP_MAX_PROJ][MOONEP_MAX_R];
 };
 
 cudaError_t launch_prefetch(const WeightArgs &a, int grid, int sms, cudaStream_t st);

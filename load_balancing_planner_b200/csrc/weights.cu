@@ -32,6 +32,36 @@ __device__ __forceinline__ int find_slot(const int32_t *row, int B, int e) {
     return (lo < B && row[lo] == e) ? lo : -1;
 }
 
+// Where the matrices live (mb = bytes per matrix).  The group: expert e is
+// row e of an [E,..] tensor, slot j = q*B + b row j of an [R*B,..] tensor.
+// One rank: its own side is a [G,..] (home experts) or [B,..] (its slots)
+// tensor at `own`; the other side is rank q's tensor peer[p][q].
+__device__ __forceinline__ char *expert_at(const WeightArgs &a, const void *own, int p, int e, size_t mb,
+                                           bool via_peers) {
+    const char *m;
+    if (a.rank < 0) {
+        m = static_cast<const char *>(own) + (size_t)e * mb;
+    } else {
+        const int G = a.d.G, q = e / G;
+        m = via_peers ? static_cast<const char *>(a.peer[p][q]) + (size_t)(e - q * G) * mb
+                      : static_cast<const char *>(own) + (size_t)(e - a.rank * G) * mb;
+    }
+    return const_cast<char *>(m);
+}
+
+__device__ __forceinline__ char *slot_at(const WeightArgs &a, const void *own, int p, int j, size_t mb,
+                                         bool via_peers) {
+    const char *m;
+    if (a.rank < 0) {
+        m = static_cast<const char *>(own) + (size_t)j * mb;
+    } else {
+        const int B = a.d.B, q = j / B;
+        m = via_peers ? static_cast<const char *>(a.peer[p][q]) + (size_t)(j - q * B) * mb
+                      : static_cast<const char *>(own) + (size_t)(j - a.rank * B) * mb;
+    }
+    return const_cast<char *>(m);
+}
+
 __device__ __forceinline__ int warp_incl_scan_w(int v) {
     const int lane = threadIdx.x & 31;
 #pragma unroll
@@ -44,8 +74,10 @@ __device__ __forceinline__ int warp_incl_scan_w(int v) {
 
 // Shared-memory slot tables: se[RB] expert or -1, nxt[RB] next slot holding
 // the same expert (-1 = last), lead[] leading slots in ascending order.
-// Returns the number of leaders, or -1 after flagging a malformed slot table.
-__device__ int build_slot_lists(const WeightArgs &a, int32_t *se, int32_t *nxt, int32_t *lead,
+// One rank's share keeps only its own slots (prefetch) or the slots holding
+// its home experts (by_home, reduce_grad).  Returns the number of leaders, or
+// -1 after flagging a malformed slot table.
+__device__ int build_slot_lists(const WeightArgs &a, int32_t *se, int32_t *nxt, int32_t *lead, bool by_home,
                                 int nthreads = kWThreads) {
     __shared__ int s_bad;
     __shared__ int s_warp[kWMaxWarps];
@@ -64,12 +96,20 @@ __device__ int build_slot_lists(const WeightArgs &a, int32_t *se, int32_t *nxt, 
         if (s % B != 0 && e >= 0) {
             const int prev = se[s - 1];
             if (prev < 0 || prev >= e) s_bad = 1;  // used slots first, ascending, distinct
+            if (prev >= 0 && prev / a.d.G != e / a.d.G) s_bad = 1;  // copies of one home group per rank
         }
     }
     __syncthreads();
     if (s_bad) {
         if (tid == 0) atomicOr(a.status, MOONEP_STATUS_BAD_PLAN);
         return -1;
+    }
+    if (a.rank >= 0) {  // whole rows are kept or dropped, so rows stay sorted
+        for (int s = tid; s < RB; s += nthreads) {
+            const int e = se[s];
+            if (e >= 0 && (by_home ? e / a.d.G != a.rank : s / B != a.rank)) se[s] = -1;
+        }
+        __syncthreads();
     }
     const int per = (RB + nthreads - 1) / nthreads;  // <= 32 (RB <= 8192)
     const int s0 = min(RB, tid * per), s1 = min(RB, s0 + per);
@@ -116,15 +156,16 @@ __device__ int build_slot_lists(const WeightArgs &a, int32_t *se, int32_t *nxt, 
     return total;
 }
 
-__global__ void __launch_bounds__(kWThreads) prefetch_kernel(WeightArgs a) {
+__global__ void __launch_bounds__(kWThreads) prefetch_kernel(const __grid_constant__ WeightArgs a) {
     pdl_wait();
     if (*a.status != 0) return;
     extern __shared__ int32_t wsm[];
     const int RB = a.d.R * a.d.B;
     int32_t *se = wsm, *nxt = wsm + RB, *lead = wsm + 2 * RB;
-    const int nlead = build_slot_lists(a, se, nxt, lead);
+    const int nlead = build_slot_lists(a, se, nxt, lead, false);
     if (nlead <= 0) return;
     const int64_t nvec = a.hhp / 8;  // bf16: 8 per 16 bytes
+    const size_t mb = (size_t)a.hhp * 2;
     const int64_t ntiles = (nvec + kWTile - 1) / kWTile;
     const int64_t units = (int64_t)a.n_proj * nlead * ntiles;
     for (int64_t u = blockIdx.x; u < units; u += gridDim.x) {
@@ -132,7 +173,7 @@ __global__ void __launch_bounds__(kWThreads) prefetch_kernel(WeightArgs a) {
         const int64_t rem = u - (int64_t)p * nlead * ntiles;
         const int s = lead[rem / ntiles];
         const int64_t t0 = (rem % ntiles) * kWTile;
-        const uint4 *src = static_cast<const uint4 *>(a.src[p]) + (int64_t)se[s] * nvec + t0;
+        const uint4 *src = reinterpret_cast<const uint4 *>(expert_at(a, a.src[p], p, se[s], mb, true)) + t0;
         uint4 x[kWVec];
 #pragma unroll
         for (int i = 0; i < kWVec; ++i) {
@@ -140,7 +181,7 @@ __global__ void __launch_bounds__(kWThreads) prefetch_kernel(WeightArgs a) {
             if (v < nvec) x[i] = __ldcs(src + i * kWThreads + threadIdx.x);
         }
         for (int j = s; j >= 0; j = nxt[j]) {
-            uint4 *dst = static_cast<uint4 *>(a.dst[p]) + (int64_t)j * nvec + t0;
+            uint4 *dst = reinterpret_cast<uint4 *>(slot_at(a, a.dst[p], p, j, mb, false)) + t0;
 #pragma unroll
             for (int i = 0; i < kWVec; ++i) {
                 const int64_t v = t0 + i * kWThreads + threadIdx.x;
@@ -158,13 +199,13 @@ __global__ void __launch_bounds__(kWThreads) prefetch_kernel(WeightArgs a) {
 constexpr int kPfStages = 3;
 constexpr uint32_t kPfTile = 32 * 1024;
 
-__global__ void __launch_bounds__(kWThreads) prefetch_bulk_kernel(WeightArgs a) {
+__global__ void __launch_bounds__(kWThreads) prefetch_bulk_kernel(const __grid_constant__ WeightArgs a) {
     pdl_wait();
     if (*a.status != 0) return;
     extern __shared__ __align__(128) int32_t wsm[];
     const int RB = a.d.R * a.d.B;
     int32_t *se = wsm, *nxt = wsm + RB, *lead = wsm + 2 * RB;
-    const int nlead = build_slot_lists(a, se, nxt, lead);
+    const int nlead = build_slot_lists(a, se, nxt, lead, false);
     if (nlead <= 0 || threadIdx.x != 0) return;
     uint8_t *stages = reinterpret_cast<uint8_t *>(wsm) + ((sizeof(int32_t) * 3 * (size_t)RB + 127) & ~(size_t)127);
     const uint32_t stage0 = smem_addr(stages);
@@ -188,8 +229,9 @@ __global__ void __launch_bounds__(kWThreads) prefetch_bulk_kernel(WeightArgs a) 
         uint64_t off;
         uint32_t n;
         piece(i, p, s, off, n);
-        bulk_load(stage0 + st * kPfTile, static_cast<const uint8_t *>(a.src[p]) + (uint64_t)se[s] * bytes_per + off,
-                  n, bar0 + 8u * st);
+        bulk_load(stage0 + st * kPfTile,
+                  reinterpret_cast<const uint8_t *>(expert_at(a, a.src[p], p, se[s], bytes_per, true)) + off, n,
+                  bar0 + 8u * st);
     };
     for (int st = 0; st < kPfStages; ++st) mbar_init(bar0 + 8u * st);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -205,7 +247,8 @@ __global__ void __launch_bounds__(kWThreads) prefetch_bulk_kernel(WeightArgs a) 
         uint32_t n;
         piece(i, p, s, off, n);
         for (int j = s; j >= 0; j = nxt[j])
-            bulk_store(static_cast<uint8_t *>(a.dst[p]) + (uint64_t)j * bytes_per + off, stage0 + st * kPfTile, n, pol);
+            bulk_store(reinterpret_cast<uint8_t *>(slot_at(a, a.dst[p], p, j, bytes_per, false)) + off,
+                       stage0 + st * kPfTile, n, pol);
         bulk_commit();
         // refill the previous unit's stage once its stores have read it
         if (i >= 1 && first + (i - 1 + kPfStages) * step < units) {
@@ -223,15 +266,16 @@ __global__ void __launch_bounds__(kWThreads) prefetch_bulk_kernel(WeightArgs a) 
 }
 
 // a.src[p] = reduce buffer [R*B, H*Hp] (read, then zeroed), a.dst[p] = grads [E, H*Hp].
-__global__ void __launch_bounds__(kWThreads) reduce_grad_kernel(WeightArgs a) {
+__global__ void __launch_bounds__(kWThreads) reduce_grad_kernel(const __grid_constant__ WeightArgs a) {
     pdl_wait();
     if (*a.status != 0) return;
     extern __shared__ int32_t wsm[];
     const int RB = a.d.R * a.d.B;
     int32_t *se = wsm, *nxt = wsm + RB, *lead = wsm + 2 * RB;
-    const int nlead = build_slot_lists(a, se, nxt, lead);
+    const int nlead = build_slot_lists(a, se, nxt, lead, true);
     if (nlead <= 0) return;
     const int64_t nvec = a.hhp / 4;  // fp32: 4 per 16 bytes
+    const size_t mb = (size_t)a.hhp * 4;
     const int64_t ntiles = (nvec + kWTile - 1) / kWTile;
     const int64_t units = (int64_t)a.n_proj * nlead * ntiles;
     const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -240,8 +284,7 @@ __global__ void __launch_bounds__(kWThreads) reduce_grad_kernel(WeightArgs a) {
         const int64_t rem = u - (int64_t)p * nlead * ntiles;
         const int s = lead[rem / ntiles];
         const int64_t t0 = (rem % ntiles) * kWTile;
-        float4 *g = static_cast<float4 *>(a.dst[p]) + (int64_t)se[s] * nvec + t0;
-        float4 *rb = static_cast<float4 *>(const_cast<void *>(a.src[p]));
+        float4 *g = reinterpret_cast<float4 *>(expert_at(a, a.dst[p], p, se[s], mb, false)) + t0;
         float4 acc[kWVec];
 #pragma unroll
         for (int i = 0; i < kWVec; ++i) {
@@ -249,7 +292,7 @@ __global__ void __launch_bounds__(kWThreads) reduce_grad_kernel(WeightArgs a) {
             acc[i] = v < nvec ? __ldcs(g + i * kWThreads + threadIdx.x) : zero;
         }
         for (int j = s; j >= 0; j = nxt[j]) {
-            const float4 *slot = rb + (int64_t)j * nvec + t0;
+            const float4 *slot = reinterpret_cast<const float4 *>(slot_at(a, a.src[p], p, j, mb, true)) + t0;
 #pragma unroll
             for (int i = 0; i < kWVec; ++i) {
                 const int64_t v = t0 + i * kWThreads + threadIdx.x;
@@ -268,7 +311,7 @@ __global__ void __launch_bounds__(kWThreads) reduce_grad_kernel(WeightArgs a) {
             if (v < nvec) __stcs(g + i * kWThreads + threadIdx.x, acc[i]);
         }
         for (int j = s; j >= 0; j = nxt[j]) {
-            float4 *slot = rb + (int64_t)j * nvec + t0;
+            float4 *slot = reinterpret_cast<float4 *>(slot_at(a, a.src[p], p, j, mb, true)) + t0;
 #pragma unroll
             for (int i = 0; i < kWVec; ++i) {
                 const int64_t v = t0 + i * kWThreads + threadIdx.x;
@@ -289,13 +332,14 @@ constexpr int kRgTile = 4096;                  // floats per piece (16 KB)
 constexpr int kRgThreads = 32 + 256;           // producer warp + 8 summing warps
 constexpr int kRgPer = kRgTile / 256;          // floats per summing thread
 
-__global__ void __launch_bounds__(kRgThreads) reduce_grad_bulk_kernel(WeightArgs a) {
+__global__ void __launch_bounds__(kRgThreads) reduce_grad_bulk_kernel(const __grid_constant__ WeightArgs a) {
     pdl_wait();
     if (*a.status != 0) return;
     extern __shared__ __align__(128) int32_t wsm[];
     const int RB = a.d.R * a.d.B;
     int32_t *se = wsm, *nxt = wsm + RB, *lead = wsm + 2 * RB;
-    const int nlead = build_slot_lists(a, se, nxt, lead, kRgThreads);
+    const int nlead = build_slot_lists(a, se, nxt, lead, true, kRgThreads);
+    const size_t mb = (size_t)a.hhp * 4;
     if (nlead <= 0) return;
     uint8_t *ring = reinterpret_cast<uint8_t *>(wsm) + ((sizeof(int32_t) * 3 * (size_t)RB + 127) & ~(size_t)127);
     const uint32_t ring0 = smem_addr(ring);
@@ -331,8 +375,7 @@ __global__ void __launch_bounds__(kRgThreads) reduce_grad_bulk_kernel(WeightArgs
                 int p, s, n;
                 int64_t off;
                 unit(i, p, s, off, n);
-                const float *g = static_cast<const float *>(a.dst[p]) + (int64_t)se[s] * a.hhp + off;
-                const float *rb = static_cast<const float *>(a.src[p]) + off;
+                const float *g = reinterpret_cast<const float *>(expert_at(a, a.dst[p], p, se[s], mb, false)) + off;
                 // the unit's pieces: its grad (j = -1), then every holder in slot order
                 for (int j = -1;;) {
                     const int k = (int)(seq % kRgRing);
@@ -341,8 +384,9 @@ __global__ void __launch_bounds__(kRgThreads) reduce_grad_bulk_kernel(WeightArgs
                         *err = 1;
                         break;
                     }
-                    bulk_load(ring0 + k * kRgTile * 4, j < 0 ? g : rb + (int64_t)j * a.hhp, (uint32_t)n * 4u,
-                              full0 + 8u * k);
+                    const float *src =
+                        j < 0 ? g : reinterpret_cast<const float *>(slot_at(a, a.src[p], p, j, mb, true)) + off;
+                    bulk_load(ring0 + k * kRgTile * 4, src, (uint32_t)n * 4u, full0 + 8u * k);
                     ++seq;
                     j = j < 0 ? s : nxt[j];
                     if (j < 0) break;
@@ -392,7 +436,7 @@ __global__ void __launch_bounds__(kRgThreads) reduce_grad_bulk_kernel(WeightArgs
             *err = 1;
             break;
         }
-        float4 *g = reinterpret_cast<float4 *>(static_cast<float *>(a.dst[p]) + (int64_t)se[s] * a.hhp + off);
+        float4 *g = reinterpret_cast<float4 *>(reinterpret_cast<float *>(expert_at(a, a.dst[p], p, se[s], mb, false)) + off);
 #pragma unroll
         for (int q = 0; q < kRgPer / 4; ++q) {
             const int idx = q * 256 + t;
@@ -400,7 +444,7 @@ __global__ void __launch_bounds__(kRgThreads) reduce_grad_bulk_kernel(WeightArgs
         }
         const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int j = s; j >= 0; j = nxt[j]) {
-            float4 *z = reinterpret_cast<float4 *>(static_cast<float *>(const_cast<void *>(a.src[p])) + (int64_t)j * a.hhp + off);
+            float4 *z = reinterpret_cast<float4 *>(reinterpret_cast<float *>(slot_at(a, a.src[p], p, j, mb, true)) + off);
 #pragma unroll
             for (int q = 0; q < kRgPer / 4; ++q) {
                 const int idx = q * 256 + t;

@@ -7,7 +7,10 @@ the rank's picks, every rank's counts: one all-gather of R x E int32
 (`gather_counts`), after which every rank derives the same layout and writes
 the slots of its own picks (`moonep_plan_rank`).  Dispatch and combine address
 the R ranks' buffers through a table of their device pointers
-(`moonep_dispatch_rank`, `moonep_combine_rank`).
+(`moonep_dispatch_rank`, `moonep_combine_rank`); the weight prefetch reads
+each slot's expert from its home rank, and the grad reduction of a home rank
+reads and zeroes the slots of every rank (`moonep_prefetch_weight_rank`,
+`moonep_reduce_grad_rank`).
 
 `RankBuffer` takes those buffers as a list of R tensors.  On a real group
 they are this rank's views of the peers' memory (peer-mapped allocations,
@@ -89,6 +92,18 @@ class RankBuffer:
         if weighted and w_nvs is None:
             raise ValueError("weighted combine needs route_weights_nvs")
         return moonep.moonep_combine_rank(self.handle, plan, list(expert_out_nvs), w_nvs, out)
+
+    def prefetch_weight(self, plan: moonep.Plan, home_weights, pools) -> None:
+        """pools[p] [B,H,H'] bf16 (this rank's slots) <- each slot's expert,
+        read from its home rank: home_weights[p][q] is rank q's [G,H,H'] bf16
+        home experts of projection p."""
+        moonep.moonep_prefetch_weight_rank(self.handle, plan, self.rank, home_weights, pools)
+
+    def reduce_grad(self, plan: moonep.Plan, grads, reduce_buffers) -> None:
+        """grads[p] [G,H,H'] fp32 (this rank's home experts) += every rank's
+        slots holding them, in (rank, slot) order; those slots are zeroed.
+        reduce_buffers[p][q] is rank q's [B,H,H'] fp32 slots."""
+        moonep.moonep_reduce_grad_rank(self.handle, plan, self.rank, grads, reduce_buffers)
 
     def destroy(self) -> None:
         if self.handle is not None:

@@ -63,6 +63,8 @@ def _load():
         "moonep_plan_rank": ([P, i32, P, P, ctypes.POINTER(PlanStruct), P], ctypes.c_int),
         "moonep_dispatch_rank": ([P, ctypes.POINTER(PlanStruct), P, P, P, P, P], ctypes.c_int),
         "moonep_combine_rank": ([P, ctypes.POINTER(PlanStruct), P, P, P, P, P], ctypes.c_int),
+        "moonep_prefetch_weight_rank": ([P, ctypes.POINTER(PlanStruct), i32, i32, P, P, i64, P], ctypes.c_int),
+        "moonep_reduce_grad_rank": ([P, ctypes.POINTER(PlanStruct), i32, i32, P, P, i64, P], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -75,7 +77,8 @@ lib = _load()
 EXPORTS = ("moonep_create", "moonep_destroy", "moonep_nvs", "moonep_get_config", "moonep_plan",
            "moonep_dispatch", "moonep_combine", "moonep_prefetch_weight", "moonep_reduce_grad",
            "moonep_read_status", "moonep_error_string", "moonep_last_error", "moonep_plan_noalloc",
-           "moonep_group_gemm", "moonep_plan_rank", "moonep_dispatch_rank", "moonep_combine_rank")
+           "moonep_group_gemm", "moonep_plan_rank", "moonep_dispatch_rank", "moonep_combine_rank",
+           "moonep_prefetch_weight_rank", "moonep_reduce_grad_rank")
 NOALLOC_SCRATCH_BYTES = 1 << 20
 
 
@@ -325,6 +328,38 @@ def moonep_reduce_grad(h: Handle, plan: Plan, grads, reduce_buffers, stream=None
         _expect(RB, (h.R, h.B, h.H, Hp), torch.float32, "reduce_buffers")
     _check(lib.moonep_reduce_grad(h.ptr, ctypes.byref(plan.struct), len(grads), _ptr_array(grads),
                                   _ptr_array(reduce_buffers), Hp, _stream(stream)), "moonep_reduce_grad")
+
+
+def _rank_weight_tables(h: Handle, own, peers, own_shape, peer_shape, dtype, names):
+    if not own or len(own) != len(peers) or any(len(row) != h.R for row in peers):
+        raise ValueError(f"one {names[0]} per projection and one {names[1]} per rank and projection")
+    Hp = own[0].shape[-1]
+    for t in own:
+        _expect(t, (*own_shape, h.H, Hp), dtype, names[0])
+    for row in peers:
+        for t in row:
+            _expect(t, (*peer_shape, h.H, Hp), dtype, names[1])
+    return _ptr_array(own), _ptr_array([t for row in peers for t in row]), Hp
+
+
+def moonep_prefetch_weight_rank(h: Handle, plan: Plan, rank: int, weights, pool, stream=None):
+    """One rank's prefetch: weights[p][q] is rank q's home experts [G,H,Hp]
+    bf16 of projection p, pool[p] this rank's slots [B,H,Hp] bf16."""
+    G = h.E // h.R
+    own, peers, Hp = _rank_weight_tables(h, list(pool), [list(r) for r in weights], (h.B,), (G,),
+                                         torch.bfloat16, ("pool", "weights"))
+    _check(lib.moonep_prefetch_weight_rank(h.ptr, ctypes.byref(plan.struct), rank, len(pool), peers, own, Hp,
+                                           _stream(stream)), "moonep_prefetch_weight_rank")
+
+
+def moonep_reduce_grad_rank(h: Handle, plan: Plan, rank: int, grads, reduce_buffers, stream=None):
+    """One home rank's reduction: grads[p] is its home experts' [G,H,Hp] fp32
+    gradients, reduce_buffers[p][q] rank q's slots [B,H,Hp] fp32."""
+    G = h.E // h.R
+    own, peers, Hp = _rank_weight_tables(h, list(grads), [list(r) for r in reduce_buffers], (G,), (h.B,),
+                                         torch.float32, ("grads", "reduce_buffers"))
+    _check(lib.moonep_reduce_grad_rank(h.ptr, ctypes.byref(plan.struct), rank, len(grads), own, peers, Hp,
+                                       _stream(stream)), "moonep_reduce_grad_rank")
 
 
 def moonep_group_gemm(h: Handle, plan: Plan, x_nvs, weights, pool=None, y_nvs=None, stream=None):

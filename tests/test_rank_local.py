@@ -227,3 +227,63 @@ def test_rank_plan_errors(cuda):
         moonep.moonep_dispatch_rank(h, p, torch.zeros((S, H), dtype=torch.bfloat16, device="cuda"), None, odd)
     assert e.value.code == moonep.ERR_ALIGN
     h.close()
+
+
+# (R, S, K, E, B, token_padding, mode, maxvio, H, Hp): bulk-copy matrices,
+# plain-vector matrices, inference with overflow (mode 1) and slots by count
+@pytest.mark.parametrize("R,S,K,E,B,tp,mode,mv,H,Hp", [
+    (8, 512, 8, 64, 8, 128, 0, 2.0, 256, 64),
+    (4, 200, 4, 32, 8, 16, 0, 1.5, 64, 32),
+    (8, 512, 8, 64, 2, 128, 1, 4.0, 256, 72),
+    (8, 512, 8, 64, 2, 128, 2, 4.0, 64, 40),
+])
+def test_rank_prefetch_and_reduce_grad_match_the_oracle(cuda, R, S, K, E, B, tp, mode, mv, H, Hp):
+    from load_balancing_planner_b200 import moonep
+    G, P = E // R, 2
+    tk, tpe, _ = problem(R, S, K, E, mv, "hot8", seed=26)
+    h = moonep.moonep_create(S, H, K, E, R, B, tp, mode=mode)
+    plans = _rank_plans(h, tk, tpe)
+    se = plans[0].slots().cpu().numpy()
+    assert (se >= 0).any()
+    gen = torch.Generator().manual_seed(26)
+    W = [torch.randn((E, H, Hp), generator=gen).to(torch.bfloat16) for _ in range(P)]
+    # every rank's home experts and slots as separate allocations
+    home = [[W[p][q * G:(q + 1) * G].cuda().contiguous() for q in range(R)] for p in range(P)]
+    pools = [[torch.full((B, H, Hp), -1, dtype=torch.int16, device="cuda").view(torch.bfloat16)
+              for _ in range(P)] for _ in range(R)]
+    for r in range(R):
+        moonep.moonep_prefetch_weight_rank(h, plans[r], r, home, pools[r])
+    torch.cuda.synchronize()
+    for p in range(P):
+        want = np.full((R * B, H * Hp), 0xFFFF, np.uint16)
+        oracle.prefetch(se, bits(W[p]).reshape(E, H * Hp), want)
+        got = np.concatenate([bits(pools[r][p]).reshape(B, H * Hp) for r in range(R)])
+        assert np.array_equal(got, want), p
+
+    Gr = [torch.randn((E, H, Hp), generator=gen) * 1e-3 for _ in range(P)]
+    RB = [torch.randn((R, B, H, Hp), generator=gen) * 1e-3 for _ in range(P)]
+    grads = [[Gr[p][q * G:(q + 1) * G].cuda().contiguous() for p in range(P)] for q in range(R)]
+    rbs = [[RB[p][q].cuda().contiguous() for q in range(R)] for p in range(P)]
+    for q in range(R):
+        moonep.moonep_reduce_grad_rank(h, plans[q], q, grads[q], rbs)
+    # the group call on the same data: same kernel, same (rank, slot) order
+    gG, gRB = [g.cuda() for g in Gr], [rb.cuda() for rb in RB]
+    moonep.moonep_reduce_grad(h, plans[0], gG, gRB)
+    torch.cuda.synchronize()
+    for p in range(P):
+        wg = Gr[p].numpy().reshape(E, H * Hp).copy()
+        wrb = RB[p].numpy().reshape(R * B, H * Hp).copy()
+        oracle.reduce_grad(se, wg, wrb)
+        got_g = np.concatenate([grads[q][p].cpu().numpy().reshape(G, H * Hp) for q in range(R)])
+        got_rb = np.concatenate([rbs[p][q].cpu().numpy().reshape(B, H * Hp) for q in range(R)])
+        assert np.array_equal(got_g.view(np.uint32), gG[p].cpu().numpy().reshape(E, -1).view(np.uint32)), p
+        assert rel_close(got_g, wg, 1e-5).all(), p
+        # consumed slots exactly +0.0, the others untouched
+        assert np.array_equal(got_rb.view(np.uint32), wrb.view(np.uint32)), p
+    # host checks: rank range, one table row per rank
+    with pytest.raises(moonep.MoonepError) as e:
+        moonep.moonep_prefetch_weight_rank(h, plans[0], R, home, pools[0])
+    assert e.value.code == moonep.ERR_SIZE
+    with pytest.raises(ValueError):
+        moonep.moonep_reduce_grad_rank(h, plans[0], 0, grads[0], [row[:R - 1] for row in rbs])
+    h.close()
