@@ -33,7 +33,7 @@ struct moonep_handle {
 // Handle workspace: [group planning][group GEMM pair table][one-rank planning]
 static size_t pair_table_offset(const Dims &d) { return (workspace_bytes(d) + 255) / 256 * 256; }
 static size_t rank_ws_offset(const Dims &d) {
-    return (pair_table_offset(d) + sizeof(int32_t) * (size_t)d.R * gemm_pair_slots(d) + 255) / 256 * 256;
+    return (pair_table_offset(d) + gemm_table_bytes(d) + 255) / 256 * 256;
 }
 
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }

@@ -109,6 +109,7 @@ cudaError_t gemm_set_smem_limit();
 int launch_group_gemm(const Dims &d, const moonep_plan_t *plan, const void *x, const void *W, const void *pool,
                       void *y, int64_t Hp, int32_t *pairs, cudaStream_t st);
 int gemm_pair_slots(const Dims &d);
+size_t gemm_table_bytes(const Dims &d);  // the pair table in the handle workspace
 
 // ---- host helpers shared by the entry points (api.cu) ----------------------
 int fail_cuda(cudaError_t e);                  // records the error text, returns MOONEP_ERR_CUDA
