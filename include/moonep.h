@@ -25,6 +25,9 @@
  *    on the host before anything is launched.  Data-dependent errors are found
  *    on the device and reported as MOONEP_STATUS_* bits in plan->status; every
  *    later call that takes that plan then does nothing.
+ *  - Every call can be captured in a CUDA graph (stream capture), the
+ *    planner's cooperative launch included; a replayed plan reads the inputs
+ *    the captured pointers hold at replay time.
  *  - Calls that share a handle must be ordered on one stream (they share the
  *    planning workspace).  Calls that overlap on the GPU and write the same
  *    caller buffers race.
