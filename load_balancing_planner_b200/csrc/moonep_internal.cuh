@@ -32,6 +32,7 @@ struct Dims {
 struct Workspace {
     int32_t *hist;                // [R*nch][E] picks per (chunk, expert)
     int32_t *cnt;                 // [2][R][E] picks per (source rank, expert), by call parity
+    int32_t *gload;               // [2][R] picks per home group (group planning), by call parity
     unsigned long long *arrive;   // planner blocks that ever reached the grid barrier
     int32_t *status;              // [2] error bits of the counting phase, by call parity
 };

@@ -32,7 +32,8 @@ __host__ __device__ static inline size_t align256(size_t b) { return (b + 255) /
 
 size_t workspace_bytes(const Dims &d) {
     return align256(sizeof(int32_t) * (size_t)d.R * d.nch * d.E) +
-           align256(sizeof(int32_t) * 2 * (size_t)d.R * d.E) + align256(4 * sizeof(uint64_t));
+           align256(sizeof(int32_t) * 2 * (size_t)d.R * d.E) + align256(sizeof(int32_t) * 2 * (size_t)d.R) +
+           align256(4 * sizeof(uint64_t));
 }
 
 void carve_workspace(const Dims &d, void *base, Workspace *ws) {
@@ -41,6 +42,8 @@ void carve_workspace(const Dims &d, void *base, Workspace *ws) {
     p += align256(sizeof(int32_t) * (size_t)d.R * d.nch * d.E);
     ws->cnt = reinterpret_cast<int32_t *>(p);
     p += align256(sizeof(int32_t) * 2 * (size_t)d.R * d.E);
+    ws->gload = reinterpret_cast<int32_t *>(p);
+    p += align256(sizeof(int32_t) * 2 * (size_t)d.R);
     ws->arrive = reinterpret_cast<unsigned long long *>(p);        // [0] blocks arrived, ever
     ws->status = reinterpret_cast<int32_t *>(p + sizeof(uint64_t));  // [2] error bits, by call parity
 }
@@ -321,6 +324,8 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
 
     __shared__ unsigned long long s_call;
     __shared__ int s_bad;
+    __shared__ int s_gl[MOONEP_MAX_R];  // this chunk's picks per home group
+    if (tid < MOONEP_MAX_R) s_gl[tid] = 0;
     if (tid == 0) {
         s_call = *reinterpret_cast<volatile unsigned long long *>(a.ws.arrive) / gridDim.x;
         s_bad = 0;
@@ -407,12 +412,17 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
             run += v;
         }
         __stcg(hrow + e, run);
-        if (run) atomicAdd(crow + e, run);
+        if (run) {
+            atomicAdd(crow + e, run);
+            if (!one_rank) atomicAdd(&s_gl[e / G], run);
+        }
     }
     bad = __reduce_or_sync(0xffffffffu, bad);
     if (lane == 0 && bad) atomicOr(&s_bad, bad);
     __syncthreads();
     if (tid == 0 && s_bad) atomicOr(a.ws.status + parity, s_bad);
+    // the group loads of this call, complete at the grid barrier
+    if (!one_rank && tid < R && s_gl[tid]) atomicAdd(a.ws.gload + (size_t)parity * R + tid, s_gl[tid]);
     PLAN_TRACE(8);
     grid_arrive(a.ws.arrive);
     // while the other blocks arrive: each pick's rank inside the chunk
@@ -430,6 +440,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
     // write to the other slot's counterpart, and the next call starts after
     // this kernel ends
     if (blockIdx.x == 0 && tid == 0) a.ws.status[parity ^ 1] = 0;
+    if (blockIdx.x == 0 && tid < R) a.ws.gload[(size_t)(parity ^ 1) * R + tid] = 0;
     {
         int32_t *next = a.ws.cnt + (size_t)(parity ^ 1) * R * E;
         const int64_t tot = (int64_t)R * E, per = (tot + gridDim.x - 1) / gridDim.x;
@@ -468,6 +479,20 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
     __shared__ int s_status, s_wmax[kPlanWarps];
 
     if (tid == kPlanThreads - 1) s_status = ld_cg(a.ws.status + parity);
+    // Group planning: the count phase summed the group loads, so one warp
+    // with no column-pass work (when E < 32 * (kPlanWarps - 1)) runs the alias
+    // chain while the others do the column pass.  One rank's planning gets
+    // its loads from the column pass below.
+    const int aw = min(kPlanWarps - 1, (E + 31) / 32);
+    if (!one_rank && w == aw) {
+        for (int h = lane; h < R; h += 32) s_L[h] = ld_cg(a.ws.gload + (size_t)parity * R + h);
+        __syncwarp();
+        AliasOut o{s_keep, s_rfrom, s_rstart, s_rlen, s_doff, s_dlist};
+        if (R <= 32)
+            alias_chain<1>(R, d.S * K, s_L, o);
+        else
+            alias_chain<2>(R, d.S * K, s_L, o);
+    }
     // Column sums of the histogram: T_e, this block's prefix (rows before its
     // own), per-rank counts (checked against the router's, written by the
     // rank's first block).
@@ -559,7 +584,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
     for (int e = tid; e < E; e += kPlanThreads) mx = max(mx, T[e]);
     mx = warp_max(mx);
     if (lane == 0) s_wmax[w] = mx;
-    for (int h = w; h < R; h += kPlanWarps) {
+    for (int h = w; one_rank && h < R; h += kPlanWarps) {
         int sum = 0;
         for (int j = lane; j < G; j += 32) sum += T[h * G + j];
         sum = warp_sum(sum);
@@ -583,7 +608,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
     // donor's gifts leave in demand-line order, so a gift starts at the
     // donor's kept count plus its distance from the donor's excess start.
     // This equals the queue-driven chain step for step.
-    if (w == 0) {
+    if (one_rank && w == 0) {
         AliasOut o{s_keep, s_rfrom, s_rstart, s_rlen, s_doff, s_dlist};
         if (R <= 32)
             alias_chain<1>(R, d.S * K, s_L, o);
