@@ -89,3 +89,32 @@ def test_buffer_layer_imports_and_names_status_bits():
     assert e.status == 5 and "outside [0, E)" in str(e) and "tokens_per_expert" in str(e)
     for name in ("dispatch", "combine", "prefetch_weight", "reduce_grad", "destroy", "check"):
         assert callable(getattr(Buffer, name))
+
+
+@pytest.mark.parametrize("S,K,E,R,tp", [(4096, 8, 256, 8, 128), (1024, 8, 64, 8, 128), (64, 2, 8, 2, 8),
+                                        (333, 3, 24, 4, 16), (40, 4, 256, 64, 8), (100, 32, 64, 2, 4)])
+def test_rank_buffer_slot_count_matches_the_oracle(S, K, E, R, tp):
+    # RankBuffer sizes peer buffers before any handle exists; its NvS must be
+    # the oracle's (both written from the same definition, separately)
+    import oracle
+    from load_balancing_planner_b200.ep import RankBuffer
+    assert RankBuffer.nvs_of(S, K, E, R, tp) == oracle.nvs(S, K, E, R, tp)
+
+
+def test_gather_counts_rejects_bad_tables_without_a_process_group():
+    import torch
+    from load_balancing_planner_b200.ep import gather_counts
+    with pytest.raises(ValueError):
+        gather_counts(torch.zeros((2, 8), dtype=torch.int32))
+    with pytest.raises(ValueError):
+        gather_counts(torch.zeros(8, dtype=torch.int64))
+
+
+def test_rank_calls_check_their_tables_before_the_device():
+    # host-side checks of the per-rank weight calls, with no handle: a NULL
+    # handle is refused before any table is read
+    from load_balancing_planner_b200 import moonep
+    P = ctypes.c_void_p
+    tab = (P * 2)()
+    assert moonep.lib.moonep_prefetch_weight_rank(None, None, 0, 1, tab, tab, 8, None) == moonep.ERR_NULL
+    assert moonep.lib.moonep_reduce_grad_rank(None, None, 0, 1, tab, tab, 8, None) == moonep.ERR_NULL
