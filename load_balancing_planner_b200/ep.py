@@ -56,8 +56,10 @@ class RankBuffer:
         self.rank, self.R = rank, num_ep_ranks
         self.S, self.H, self.K, self.E, self.B = S, H, K, E, self.handle.B
         self.nvs = self.handle.nvs
-        self.hidden_nvs = list(hidden_nvs)
-        self.route_weights_nvs = None if route_weights_nvs is None else list(route_weights_nvs)
+        # checked and marshalled once: the per-layer calls pass the tables
+        self.hidden_nvs = moonep.PeerTable(hidden_nvs, (self.nvs, H), torch.bfloat16, "hidden_nvs[q]")
+        self.route_weights_nvs = None if route_weights_nvs is None else moonep.PeerTable(
+            route_weights_nvs, (self.nvs,), torch.float32, "route_weights_nvs[q]")
 
     @staticmethod
     def nvs_of(S: int, K: int, E: int, num_ep_ranks: int, token_padding: int = 128) -> int:
@@ -83,15 +85,17 @@ class RankBuffer:
         w_nvs = self.route_weights_nvs if route_weights is not None else None
         moonep.moonep_dispatch_rank(self.handle, plan, hidden, route_weights, self.hidden_nvs, w_nvs)
 
-    def combine(self, plan: moonep.Plan, expert_out_nvs, weighted: bool = True, out=None):
+    def combine(self, plan: moonep.Plan, expert_out_nvs=None, weighted: bool = True, out=None):
         """out [S,H] = bf16(sum_k w_k * y[slot of (t,k)]) over this rank's
-        tokens, reading `expert_out_nvs` (the R ranks' [NvS,H] outputs, a list
-        like hidden_nvs) and, when weighted, the route weights that dispatch
-        placed.  Returns (out, gathered_weights [S,K] or None)."""
+        tokens, reading `expert_out_nvs` (the R ranks' [NvS,H] outputs: a list
+        or a moonep.PeerTable; None reads the dispatch buffers themselves)
+        and, when weighted, the route weights that dispatch placed.  Returns
+        (out, gathered_weights [S,K] or None)."""
         w_nvs = self.route_weights_nvs if weighted else None
         if weighted and w_nvs is None:
             raise ValueError("weighted combine needs route_weights_nvs")
-        return moonep.moonep_combine_rank(self.handle, plan, list(expert_out_nvs), w_nvs, out)
+        y = self.hidden_nvs if expert_out_nvs is None else expert_out_nvs
+        return moonep.moonep_combine_rank(self.handle, plan, y, w_nvs, out)
 
     def prefetch_weight(self, plan: moonep.Plan, home_weights, pools) -> None:
         """pools[p] [B,H,H'] bf16 (this rank's slots) <- each slot's expert,

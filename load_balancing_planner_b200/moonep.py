@@ -228,8 +228,9 @@ def moonep_plan_rank(h: Handle, rank: int, topk, counts_all, plan: Plan | None =
 def moonep_dispatch_rank(h: Handle, plan: Plan, hidden, route_weights, hidden_nvs, route_weights_nvs=None,
                          stream=None):
     """Scatter one rank's rows hidden [S,H] (and route_weights [S,K]) into the
-    R ranks' buffers: hidden_nvs is a list of R [NvS,H] bf16 tensors,
-    route_weights_nvs None or a list of R [NvS] fp32 tensors."""
+    R ranks' buffers: hidden_nvs is a list (or PeerTable) of R [NvS,H] bf16
+    tensors, route_weights_nvs None or a list (or PeerTable) of R [NvS] fp32
+    tensors."""
     _rank_plan(plan, "moonep_dispatch_rank")
     _expect(hidden, (h.S, h.H), torch.bfloat16, "hidden")
     _expect(route_weights, (h.S, h.K), torch.float32, "route_weights")
@@ -256,14 +257,43 @@ def moonep_combine_rank(h: Handle, plan: Plan, hidden_nvs, route_weights_nvs=Non
     return out, gathered_weights
 
 
-def _rank_tables(h: Handle, hidden_nvs, route_weights_nvs):
-    if len(hidden_nvs) != h.R or (route_weights_nvs is not None and len(route_weights_nvs) != h.R):
+class PeerTable:
+    """The R ranks' same-shaped tensors as one table of device pointers,
+    checked once.  Pass it wherever a per-rank call takes a list of R
+    tensors: the call then skips the per-tensor checks and the marshalling.
+    The table keeps the tensors alive; their storage must not move."""
+
+    def __init__(self, tensors, shape, dtype, name="table"):
+        self.tensors = list(tensors)
+        for t in self.tensors:
+            _expect(t, shape, dtype, name)
+        self.arr = _ptr_array(self.tensors)
+        self.shape, self.dtype, self.name = tuple(shape), dtype, name
+
+    def __len__(self):
+        return len(self.tensors)
+
+    def __getitem__(self, i):
+        return self.tensors[i]
+
+
+def _table(h: Handle, x, shape, dtype, name):
+    if x is None:
+        return None
+    if isinstance(x, PeerTable):
+        if len(x) != h.R or x.shape != tuple(shape) or x.dtype != dtype:
+            raise ValueError(f"{name}: a table of {h.R} {tuple(shape)} {dtype} tensors expected")
+        return x.arr
+    if len(x) != h.R:
         raise ValueError("one buffer per rank")
-    for b in hidden_nvs:
-        _expect(b, (h.nvs, h.H), torch.bfloat16, "hidden_nvs[q]")
-    for b in route_weights_nvs or ():
-        _expect(b, (h.nvs,), torch.float32, "route_weights_nvs[q]")
-    return _ptr_array(hidden_nvs), (_ptr_array(route_weights_nvs) if route_weights_nvs is not None else None)
+    for b in x:
+        _expect(b, shape, dtype, name)
+    return _ptr_array(x)
+
+
+def _rank_tables(h: Handle, hidden_nvs, route_weights_nvs):
+    return (_table(h, hidden_nvs, (h.nvs, h.H), torch.bfloat16, "hidden_nvs[q]"),
+            _table(h, route_weights_nvs, (h.nvs,), torch.float32, "route_weights_nvs[q]"))
 
 
 def moonep_dispatch(h: Handle, plan: Plan, hidden, route_weights=None, hidden_nvs=None,

@@ -163,12 +163,19 @@ def test_rank_path_roundtrip_through_rank_buffer(cuda):
         p = rb.plan(torch.from_numpy(np.ascontiguousarray(tk[r])).cuda(), counts_all=c)
         rb.dispatch(p, x[r].contiguous(), w[r].contiguous())
         plans.append(p)
+    from load_balancing_planner_b200 import moonep
+    table = moonep.PeerTable(bufs, (nvs, H), torch.bfloat16)
     for r, rb in enumerate(ranks):
         out, gw = rb.combine(plans[r], bufs, weighted=False)
         assert gw is None
         assert torch.equal(out, (x[r].float() * K).to(torch.bfloat16))
+        # the same through a table checked once, and through the rank's own tables
+        assert torch.equal(rb.combine(plans[r], table, weighted=False)[0], out)
+        assert torch.equal(rb.combine(plans[r], weighted=False)[0], out)
         _, gw = rb.combine(plans[r], bufs)
         assert torch.equal(gw, w[r])  # each slot's weight travelled with its row
+    with pytest.raises(ValueError):  # a table of the wrong tensors
+        ranks[0].combine(plans[0], moonep.PeerTable(wbufs, (nvs,), torch.float32))
     for rb in ranks:
         rb.destroy()
 
