@@ -95,12 +95,12 @@ def copy_source_hash():
 
 def recorded_traffic(kernel):
     """DRAM bytes per launch of `kernel` at the training shape, from the ncu
-    record in profiles/dram_traffic_train.md -- only if that record was taken
+    record in profiles/dram_traffic_train.txt -- only if that record was taken
     on the current source of the copy kernels (hash match), else None."""
     import re
     try:
         sha = copy_source_hash()
-        with open(os.path.join(ROOT, "profiles", "dram_traffic_train.md")) as f:
+        with open(os.path.join(ROOT, "profiles", "dram_traffic_train.txt")) as f:
             for line in f:
                 m = re.search(r"traffic: kernel=(\w+) bytes_per_launch=(\d+) copy_src_sha256=(\w+)", line)
                 if m and m.group(1) == kernel and m.group(3) == sha:
