@@ -47,6 +47,8 @@ def lib():
         L.oracle_double_to_bf16.restype = ctypes.c_uint16
         L.oracle_plan.argtypes = [i, i, i, i, i, i, i, P, P, P, P, P, P, P, P, P]
         L.oracle_plan.restype = i
+        L.oracle_plan_rank.argtypes = [i, i, i, i, i, i, i, i, P, P, P, P, P, P, P, P]
+        L.oracle_plan_rank.restype = i
         L.oracle_dispatch.argtypes = [i, i, i, i, P, P, P, P, P]
         L.oracle_dispatch.restype = None
         L.oracle_combine.argtypes = [i, i, i, i, P, P, P, P, P]
@@ -100,6 +102,30 @@ def plan(topk, E: int, B: int, tp: int, mode: int = 0, tpe=None) -> dict:
     out["status"] = int(st)
     out["maxvio"] = float(out["maxvio"][0])
     out["nvs"] = nvs(S, K, E, R, tp) if st != STATUS_BAD_ARGS else 0
+    return out
+
+
+def plan_rank(topk, counts, rank: int, E: int, B: int, tp: int, mode: int = 0) -> dict:
+    """One rank's share of the plan from its own picks ``topk`` [S, K] and
+    every rank's counts ``counts`` [R, E]: dst [S, K] and the group layout."""
+    topk = _c(topk, np.int32)
+    counts = _c(counts, np.int32)
+    S, K = topk.shape
+    R = counts.shape[0]
+    NR = E + B
+    out = dict(
+        dst=np.full((S, K), -1, np.int32),
+        cu_seqlens=np.zeros((R, NR), np.int32),
+        row_counts=np.zeros((R, NR), np.int32),
+        slot_expert=np.full((R, max(B, 0)), -1, np.int32),
+        maxvio=np.zeros(1, np.float32),
+        assign=np.zeros((R, 4), np.int32),
+    )
+    st = lib().oracle_plan_rank(R, S, K, E, B, tp, mode, rank, _p(topk), _p(counts), _p(out["dst"]),
+                                _p(out["cu_seqlens"]), _p(out["row_counts"]), _p(out["slot_expert"]),
+                                _p(out["maxvio"]), _p(out["assign"]))
+    out["status"] = int(st)
+    out["maxvio"] = float(out["maxvio"][0])
     return out
 
 

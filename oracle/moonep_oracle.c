@@ -58,6 +58,11 @@
  *  7. NvS = roundup(C + 2*G*(tp-1), tp): at most G home rows plus G received
  *     rows are non-empty.  [reading]
  *  8. dst[r,t,k] = dest_rank*NvS + row start + position inside the row.
+ *
+ * oracle_plan_rank gives one rank's share: steps 1-6 from the gathered counts
+ * alone, and step 8 for the rank's own picks in closed form (a pick's place
+ * in its group sequence follows from the counts of the ranks before it).
+ * The tests check it against oracle_plan's walk on every rank.
  */
 #include <math.h>
 #include <stdint.h>
@@ -111,56 +116,33 @@ uint16_t oracle_double_to_bf16(double x)
 
 /* ---- plan --------------------------------------------------------------- */
 
-/*
- * Inputs: topk [R,S,K] int32 (expert ids), tpe [R,E] int32 or NULL (the
- * router's local counts, checked against the picks).  mode 0 = training
- * (B >= E/R), 1 = inference, 2 = inference with slots by token count.
- * Outputs (caller-allocated): dst [R,S,K], cu_seqlens [R,E+B],
- * row_counts [R,E+B], slot_expert [R,B] (-1 = unused), counts [R,E],
- * maxvio [1], assign [R,4] = {kept, donor group or -1, received start in the
- * donor's group sequence, received length}.
- * Returns 0 or a bitmask of ORC_* errors; on error the outputs other than
- * counts are not written.
- */
-int oracle_plan(int R, int S, int K, int E, int B, int tp, int mode,
-                const int32_t *topk, const int32_t *tpe,
-                int32_t *dst, int32_t *cu_seqlens, int32_t *row_counts,
-                int32_t *slot_expert, int32_t *counts, float *maxvio,
-                int32_t *assign)
+/* What step 8 needs from the layout (see plan_layout). */
+struct layout {
+    int64_t *T, *L, *keep, *estart, *don_amt, *don_start;
+    int *don_from, *don_to;
+    int ndon;
+};
+
+static void layout_free(struct layout *y)
 {
-    if (R < 1 || S < 1 || K < 1 || E < 1 || E % R || K > E || B < 0 || tp < 1)
-        return ORC_BAD_ARGS;
+    free(y->T); free(y->L); free(y->keep); free(y->estart); free(y->don_amt);
+    free(y->don_start); free(y->don_from); free(y->don_to);
+}
+
+/*
+ * Steps 1 (loads, maxvio) to 6 from the per-rank counts [R,E] alone: the
+ * alias chain, the kept prefixes and donated ranges, the rows of every rank
+ * and their padded end offsets.  Writes maxvio, assign, row_counts,
+ * slot_expert and cu_seqlens; returns in *y what step 8 needs (free with
+ * layout_free).  The counts must hold S*K picks per rank.
+ */
+static void plan_layout(int R, int S, int K, int E, int B, int tp, int mode, const int32_t *counts,
+                        float *maxvio, int32_t *assign, int32_t *row_counts, int32_t *slot_expert,
+                        int32_t *cu_seqlens, struct layout *y)
+{
     const int G = E / R;
-    if (mode < 0 || mode > 2 || (mode == 0 && B < G)) return ORC_BAD_ARGS;
     const int64_t C = (int64_t)S * K;
     const int NR = E + B; /* rows per rank */
-    const int64_t NvS = oracle_nvs(S, K, E, R, tp);
-    int status = 0;
-
-    /* validation: ids in [0,E), no expert twice within one token */
-    for (int r = 0; r < R; r++)
-        for (int t = 0; t < S; t++) {
-            const int32_t *tok = topk + ((int64_t)r * S + t) * K;
-            for (int k = 0; k < K; k++) {
-                int e = tok[k];
-                if (e < 0 || e >= E) { status |= ORC_BAD_EXPERT; continue; }
-                for (int k2 = 0; k2 < k; k2++)
-                    if (tok[k2] == e) status |= ORC_DUP_EXPERT;
-            }
-        }
-
-    /* step 1: counts over the valid picks */
-    memset(counts, 0, sizeof(int32_t) * (size_t)R * E);
-    for (int r = 0; r < R; r++)
-        for (int64_t i = 0; i < C; i++) {
-            int e = topk[(int64_t)r * C + i];
-            if (e >= 0 && e < E) counts[(int64_t)r * E + e]++;
-        }
-    if (tpe)
-        for (int64_t i = 0; i < (int64_t)R * E; i++)
-            if (tpe[i] != counts[i]) status |= ORC_COUNT_MISMATCH;
-    if (status) return status;
-
     int64_t *T = calloc(E, sizeof(int64_t));
     int64_t *L = calloc(R, sizeof(int64_t));
     for (int e = 0; e < E; e++) {
@@ -285,6 +267,67 @@ int oracle_plan(int R, int S, int K, int E, int B, int tp, int mode,
         }
     }
 
+    free(rx_n); free(rx_e); free(largeq); free(smallq); free(cur);
+    y->T = T; y->L = L; y->keep = keep; y->estart = estart; y->don_amt = don_amt;
+    y->don_start = don_start; y->don_from = don_from; y->don_to = don_to; y->ndon = ndon;
+}
+
+/*
+ * Inputs: topk [R,S,K] int32 (expert ids), tpe [R,E] int32 or NULL (the
+ * router's local counts, checked against the picks).  mode 0 = training
+ * (B >= E/R), 1 = inference, 2 = inference with slots by token count.
+ * Outputs (caller-allocated): dst [R,S,K], cu_seqlens [R,E+B],
+ * row_counts [R,E+B], slot_expert [R,B] (-1 = unused), counts [R,E],
+ * maxvio [1], assign [R,4] = {kept, donor group or -1, received start in the
+ * donor's group sequence, received length}.
+ * Returns 0 or a bitmask of ORC_* errors; on error the outputs other than
+ * counts are not written.
+ */
+int oracle_plan(int R, int S, int K, int E, int B, int tp, int mode,
+                const int32_t *topk, const int32_t *tpe,
+                int32_t *dst, int32_t *cu_seqlens, int32_t *row_counts,
+                int32_t *slot_expert, int32_t *counts, float *maxvio,
+                int32_t *assign)
+{
+    if (R < 1 || S < 1 || K < 1 || E < 1 || E % R || K > E || B < 0 || tp < 1)
+        return ORC_BAD_ARGS;
+    const int G = E / R;
+    if (mode < 0 || mode > 2 || (mode == 0 && B < G)) return ORC_BAD_ARGS;
+    const int64_t C = (int64_t)S * K;
+    const int NR = E + B; /* rows per rank */
+    const int64_t NvS = oracle_nvs(S, K, E, R, tp);
+    int status = 0;
+
+    /* validation: ids in [0,E), no expert twice within one token */
+    for (int r = 0; r < R; r++)
+        for (int t = 0; t < S; t++) {
+            const int32_t *tok = topk + ((int64_t)r * S + t) * K;
+            for (int k = 0; k < K; k++) {
+                int e = tok[k];
+                if (e < 0 || e >= E) { status |= ORC_BAD_EXPERT; continue; }
+                for (int k2 = 0; k2 < k; k2++)
+                    if (tok[k2] == e) status |= ORC_DUP_EXPERT;
+            }
+        }
+
+    /* step 1: counts over the valid picks */
+    memset(counts, 0, sizeof(int32_t) * (size_t)R * E);
+    for (int r = 0; r < R; r++)
+        for (int64_t i = 0; i < C; i++) {
+            int e = topk[(int64_t)r * C + i];
+            if (e >= 0 && e < E) counts[(int64_t)r * E + e]++;
+        }
+    if (tpe)
+        for (int64_t i = 0; i < (int64_t)R * E; i++)
+            if (tpe[i] != counts[i]) status |= ORC_COUNT_MISMATCH;
+    if (status) return status;
+
+    struct layout y;
+    plan_layout(R, S, K, E, B, tp, mode, counts, maxvio, assign, row_counts, slot_expert, cu_seqlens, &y);
+    int64_t *keep = y.keep, *don_start = y.don_start, *don_amt = y.don_amt;
+    int *don_from = y.don_from, *don_to = y.don_to;
+    const int ndon = y.ndon;
+
     /* step 8: walk each group sequence in order and place every pick */
     int32_t *fill = calloc((size_t)R * NR, sizeof(int32_t));
     for (int h = 0; h < R; h++) {
@@ -313,10 +356,92 @@ int oracle_plan(int R, int S, int K, int E, int B, int tp, int mode,
                     }
     }
 
-    free(rx_n); free(rx_e);
-    free(fill); free(estart); free(don_start); free(keep); free(don_amt);
-    free(don_to); free(don_from); free(largeq); free(smallq); free(cur);
-    free(L); free(T);
+    free(fill);
+    layout_free(&y);
+    return 0;
+}
+
+/*
+ * One rank's share of the plan, from what a rank of a real EP group holds:
+ * its own picks topk [S,K] and every rank's counts [R,E] (gathered; README
+ * "dispatch fwd" gives each rank its local tokens_per_expert).  The layout
+ * (steps 1-6) needs only the counts.  In step 2's order, a pick of expert e
+ * at token t of this rank sits at
+ *   g = estart[e] + sum_{q < rank} counts[q][e] + (its rank among this
+ *       rank's picks of e, in token order)
+ * of its group sequence; step 8 puts it at row position g - (the first g of
+ * that row's run of e), a closed form of the walk oracle_plan performs.
+ * Outputs: dst [S,K] for this rank's picks; cu_seqlens, row_counts,
+ * slot_expert, maxvio and assign of the whole group, as oracle_plan writes
+ * them.  Returns 0 or ORC_* bits: BAD_EXPERT / DUP_EXPERT in the rank's
+ * picks; COUNT_MISMATCH when row `rank` of the counts differs from the
+ * picks, or a row holds a negative count or does not sum to S*K.
+ */
+int oracle_plan_rank(int R, int S, int K, int E, int B, int tp, int mode, int rank,
+                     const int32_t *topk, const int32_t *counts,
+                     int32_t *dst, int32_t *cu_seqlens, int32_t *row_counts,
+                     int32_t *slot_expert, float *maxvio, int32_t *assign)
+{
+    if (R < 1 || S < 1 || K < 1 || E < 1 || E % R || K > E || B < 0 || tp < 1 || rank < 0 || rank >= R)
+        return ORC_BAD_ARGS;
+    const int G = E / R;
+    if (mode < 0 || mode > 2 || (mode == 0 && B < G)) return ORC_BAD_ARGS;
+    const int64_t C = (int64_t)S * K;
+    const int NR = E + B;
+    const int64_t NvS = oracle_nvs(S, K, E, R, tp);
+    int status = 0;
+
+    int64_t *mine = calloc(E, sizeof(int64_t));
+    for (int t = 0; t < S; t++) {
+        const int32_t *tok = topk + (int64_t)t * K;
+        for (int k = 0; k < K; k++) {
+            int e = tok[k];
+            if (e < 0 || e >= E) { status |= ORC_BAD_EXPERT; continue; }
+            for (int k2 = 0; k2 < k; k2++)
+                if (tok[k2] == e) status |= ORC_DUP_EXPERT;
+            mine[e]++;
+        }
+    }
+    for (int e = 0; e < E; e++)
+        if (mine[e] != counts[(int64_t)rank * E + e]) status |= ORC_COUNT_MISMATCH;
+    for (int q = 0; q < R; q++) {
+        int64_t sum = 0;
+        for (int e = 0; e < E; e++) {
+            int32_t v = counts[(int64_t)q * E + e];
+            if (v < 0) status |= ORC_COUNT_MISMATCH;
+            sum += v;
+        }
+        if (sum != C) status |= ORC_COUNT_MISMATCH;
+    }
+    free(mine);
+    if (status) return status;
+
+    struct layout y;
+    plan_layout(R, S, K, E, B, tp, mode, counts, maxvio, assign, row_counts, slot_expert, cu_seqlens, &y);
+    int64_t *seen = calloc(E, sizeof(int64_t));
+    for (int t = 0; t < S; t++)
+        for (int k = 0; k < K; k++) {
+            const int e = topk[(int64_t)t * K + k], h = e / G;
+            int64_t pre = 0;
+            for (int q = 0; q < rank; q++) pre += counts[(int64_t)q * E + e];
+            const int64_t g = y.estart[e] + pre + seen[e]++;
+            int dest = h, row = e;
+            int64_t first = y.estart[e];
+            if (g >= y.keep[h]) {
+                for (int j = 0; j < y.ndon; j++)
+                    if (y.don_from[j] == h && g >= y.don_start[j] && g < y.don_start[j] + y.don_amt[j]) {
+                        dest = y.don_to[j];
+                        first = y.estart[e] > y.don_start[j] ? y.estart[e] : y.don_start[j];
+                    }
+                for (int b = 0; b < B; b++)
+                    if (slot_expert[(int64_t)dest * B + b] == e) row = E + b;
+            }
+            const int64_t ri = (int64_t)dest * NR + row;
+            const int64_t row_start = cu_seqlens[ri] - pad_up(row_counts[ri], tp);
+            dst[(int64_t)t * K + k] = (int32_t)(dest * NvS + row_start + (g - first));
+        }
+    free(seen);
+    layout_free(&y);
     return 0;
 }
 

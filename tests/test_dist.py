@@ -81,6 +81,12 @@ def _gather_worker(rank, world, port, q):
         # the oracle accepts as the router counts of the group's picks
         ok = np.array_equal(table, synth.local_counts(tk, 16))
         st = oracle.plan(tk, 16, 8, 8, 0, table)["status"]
+        # this rank's share from its own picks and the gathered table equals
+        # its slice of the plan of the whole group
+        mine = oracle.plan_rank(tk[rank], table, rank, 16, 8, 8, 0)
+        group = oracle.plan(tk, 16, 8, 8, 0)
+        ok = ok and mine["status"] == 0 and np.array_equal(mine["dst"], group["dst"][rank]) and \
+            np.array_equal(mine["cu_seqlens"], group["cu_seqlens"])
         q.put((rank, bool(ok), int(st), table.tobytes()))
     finally:
         dist.barrier()

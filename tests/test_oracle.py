@@ -517,3 +517,51 @@ def test_bruteforce_min_copies_tiny():
         gaps.append(mine - best)
     gaps = np.array(gaps)
     assert gaps.max() <= 1  # observed on this tiny space; reported, not a page claim
+
+
+# ------------------------------------------------ one rank's share of the plan
+@pytest.mark.parametrize("R,S,K,E,B,tp,mode,mv,profile", [
+    (8, 1024, 8, 64, 8, 128, 0, 2.0, "zipf"),
+    (8, 1024, 8, 64, 8, 128, 0, 0.0, "hot8"),
+    (3, 1000, 3, 24, 8, 16, 0, 1.5, "hot8"),
+    (4, 333, 3, 24, 0, 16, 1, 1.5, "hot8"),
+    (8, 512, 8, 64, 2, 128, 1, 4.0, "hot8"),
+    (8, 512, 8, 64, 2, 128, 2, 4.0, "hot8"),
+    (2, 100, 32, 64, 32, 4, 0, 0.5, "zipf"),
+    (16, 64, 4, 64, 4, 8, 0, 6.0, "hot8"),
+])
+def test_rank_share_is_the_slice_of_the_group_plan(R, S, K, E, B, tp, mode, mv, profile):
+    # The group plan walks every group sequence with all ranks' picks; a
+    # rank's share places its own picks from the counts in closed form.  The
+    # two must agree on every rank, which is what lets each rank of a real
+    # group plan for itself after one all-gather of the counts.
+    tk, _, _ = synth.routing(R, S, K, E, mv, profile, seed=17)
+    cnt = synth.local_counts(tk, E)
+    want = oracle.plan(tk, E, B, tp, mode, cnt)
+    assert want["status"] == 0
+    for r in range(R):
+        got = oracle.plan_rank(tk[r], cnt, r, E, B, tp, mode)
+        assert got["status"] == 0
+        assert np.array_equal(got["dst"], want["dst"][r]), r
+        for k in ("cu_seqlens", "row_counts", "slot_expert", "assign"):
+            assert np.array_equal(got[k], want[k]), (r, k)
+        assert np.float32(got["maxvio"]) == np.float32(want["maxvio"])
+
+
+def test_rank_share_refuses_inconsistent_counts():
+    R, S, K, E, B, tp = 4, 64, 4, 16, 4, 8
+    tk, _, _ = synth.routing(R, S, K, E, 1.0, "hot8", seed=18)
+    cnt = synth.local_counts(tk, E)
+    moved = cnt.copy()
+    e0, e1 = int(np.argmax(moved[1])), int(np.argmin(moved[1]))
+    moved[1, e0] -= 1
+    moved[1, e1] += 1
+    assert oracle.plan_rank(tk[1], moved, 1, E, B, tp)["status"] == oracle.STATUS_COUNT_MISMATCH
+    assert oracle.plan_rank(tk[0], moved, 0, E, B, tp)["status"] == 0  # rank 0 sees only its own row
+    short = cnt.copy()
+    short[2, int(np.argmax(short[2]))] -= 1
+    assert oracle.plan_rank(tk[0], short, 0, E, B, tp)["status"] == oracle.STATUS_COUNT_MISMATCH
+    bad = tk[3].copy()
+    bad[0, 0] = E
+    assert oracle.plan_rank(bad, cnt, 3, E, B, tp)["status"] & oracle.STATUS_BAD_EXPERT
+    assert oracle.plan_rank(tk[0], cnt, R, E, B, tp)["status"] == oracle.STATUS_BAD_ARGS

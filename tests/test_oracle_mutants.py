@@ -57,6 +57,11 @@ MUTANTS = {
     "slots by count take the fewest picks": (
         "if (rx_n[m] > rx_n[j] || (rx_n[m] == rx_n[j] && m < j)) better++;",
         "if (rx_n[m] < rx_n[j] || (rx_n[m] == rx_n[j] && m < j)) better++;"),
+    "rank share counts its own rank in the prefix": (
+        "for (int q = 0; q < rank; q++) pre += counts[(int64_t)q * E + e];",
+        "for (int q = 0; q <= rank; q++) pre += counts[(int64_t)q * E + e];"),
+    "rank share positions from the expert start only": (
+        "first = y.estart[e] > y.don_start[j] ? y.estart[e] : y.don_start[j];", "first = y.estart[e];"),
     "slots by count break ties to the higher id": (
         "if (rx_n[m] > rx_n[j] || (rx_n[m] == rx_n[j] && m < j)) better++;",
         "if (rx_n[m] > rx_n[j] || (rx_n[m] == rx_n[j] && m > j)) better++;"),

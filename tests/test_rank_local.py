@@ -60,6 +60,8 @@ def test_rank_plans_match_the_group_plan_of_the_oracle(cuda, case):
         assert moonep.moonep_read_status(p) == 0, r
         assert p.dst.shape == (S, K)
         assert np.array_equal(p.dst.cpu().numpy(), want["dst"][r]), f"dst of rank {r}"
+        mine = oracle.plan_rank(tk[r], tpe, r, E, B, tp, mode)  # the rank's share, placed in closed form
+        assert mine["status"] == 0 and np.array_equal(mine["dst"], want["dst"][r])
         for k in PLAN_WHOLE:
             g = getattr(p, k).cpu().numpy()
             if k == "slot_expert":
