@@ -118,3 +118,38 @@ def test_rank_calls_check_their_tables_before_the_device():
     tab = (P * 2)()
     assert moonep.lib.moonep_prefetch_weight_rank(None, None, 0, 1, tab, tab, 8, None) == moonep.ERR_NULL
     assert moonep.lib.moonep_reduce_grad_rank(None, None, 0, 1, tab, tab, 8, None) == moonep.ERR_NULL
+
+
+C_CALLER = r"""
+#include <stdio.h>
+#include <string.h>
+#include "moonep.h"
+int main(void) {
+    moonep_config_t c = {64, 128, 2, 10, 4, 4, 8, 0, 0};  /* E % R != 0 */
+    moonep_handle_t h = (moonep_handle_t)0;
+    if (moonep_create(&c, &h) != MOONEP_ERR_CONFIG || h) return 1;
+    if (strcmp(moonep_error_string(MOONEP_ERR_CONFIG), "configuration rejected") != 0) return 2;
+    if (moonep_plan_rank(0, 0, 0, 0, 0, 0) != MOONEP_ERR_NULL) return 3;
+    if (moonep_dispatch_rank(0, 0, 0, 0, 0, 0, 0) != MOONEP_ERR_NULL) return 4;
+    if (moonep_destroy(0) != MOONEP_OK) return 5;
+    puts("ok");
+    return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_the_library_links_from_c(tmp_path):
+    # the boundary is a C ABI: a C99 program includes the header (pedantic,
+    # warnings as errors), links the library and calls it, with no GPU needed
+    import subprocess
+    from load_balancing_planner_b200 import build
+    lib = build.build()
+    src = tmp_path / "caller.c"
+    src.write_text(C_CALLER)
+    exe = tmp_path / "caller"
+    libdir = os.path.dirname(lib)
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I",
+                    os.path.join(ROOT, "include"), "-o", str(exe), str(src), "-L", libdir, "-lmoonep",
+                    f"-Wl,-rpath,{libdir}"], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0 and out.stdout.strip() == "ok", (out.returncode, out.stdout, out.stderr)
