@@ -12,18 +12,23 @@
 // One cooperative launch, one block per (source rank, chunk of `ct` tokens),
 // all blocks resident:
 //   A. count: the chunk's picks go to shared memory; each warp ranks its runs
-//      of 32 picks per expert with match_any/popc (token order), which also
-//      finds an expert picked twice by one token; per-warp counts are scanned
-//      into the chunk's histogram row (global) and every pick's stable rank
-//      inside the chunk.
+//      of 32 picks per expert with lane masks (shared-memory atomicOr, then
+//      popc below the lane: token order), which also finds an expert picked
+//      twice by one token; per-warp counts are scanned into the chunk's
+//      histogram row (global), its per-rank counts and its picks per home
+//      group, and every pick gets its stable rank inside the chunk.
 //   -- grid barrier: one 64-bit arrive counter that only grows; bounded spin.
-//   B. layout, computed by every block from the histogram (no second
-//      barrier): T_e, loads, maxvio, the alias chain (one warp, in closed form
-//      over prefix sums of deficits and excesses), expert starts, and per rank
-//      a compact row table with inclusive running sums.
+//   B. layout, computed by every block from the histograms (no second
+//      barrier): T_e, maxvio, the alias chain (one warp, in closed form over
+//      prefix sums of deficits and excesses; it runs on a spare warp during
+//      the column pass, from the group loads the count phase summed), expert
+//      starts, and per rank a compact row table with inclusive running sums.
 //   C. every block writes a slice of cu_seqlens / row_counts / slot_expert,
 //      then dst for its own picks from per-expert bases (one shared-memory
 //      read per pick in the common case).
+// One rank's share (src_rank >= 0) runs the same kernel over that rank's
+// chunks only: the other ranks' counts come from the gathered table, which
+// every block validates first, and the alias chain follows the column pass.
 #include "moonep_internal.cuh"
 
 namespace moonep {
