@@ -108,3 +108,23 @@ def test_two_rank_count_gather_gloo():
     assert ok0 and ok1
     assert st0 == st1 == 0
     assert t0 == t1, "every rank holds the same table"
+
+
+def test_reference_arm_prints_one_contract_line():
+    # `bench.py --impl reference` (the CPU oracle, the base contract's
+    # reference arm) prints one JSON line with the keys the driver reads
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--config", "zipf", "--steps", "1",
+                          "--warmup", "3"], cwd=root, capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stderr[-500:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for k in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+              "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert k in d, k
+    assert d["impl"] == "reference" and d["value"] > 0 and d["steps"] == 1 and d["warmup"] == 3
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
