@@ -48,6 +48,8 @@ struct PlanArgs {
     const int32_t *counts_all;  // [R,E] every rank's counts (src_rank >= 0)
     moonep_plan_t plan;
     Workspace ws;
+    uint32_t polls;     // grid-barrier poll limit (kBarrierPolls unless a test lowers it)
+    uint32_t withheld;  // arrivals the barrier waits for beyond the grid (0; a test hook sets it)
 };
 
 size_t plan_smem_bytes(const Dims &d);

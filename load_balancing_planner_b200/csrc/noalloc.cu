@@ -63,6 +63,8 @@ extern "C" int moonep_plan_noalloc(const moonep_config_t *cfg, const int32_t *to
     a.src_rank = -1;
     a.counts_all = nullptr;
     a.plan = *plan;
+    a.polls = kBarrierPolls;
+    a.withheld = 0;
     carve_workspace(d, base, &a.ws);
     // The array keeps the previous call's contents.  What must start at zero
     // -- the per-rank count tables, the barrier counter and the error slots,

@@ -135,7 +135,9 @@ __device__ __forceinline__ int pad_to(int n, int tp) { return n ? (n + tp - 1) /
 // wait so a block can do local work in between.  The counter only grows: at
 // kernel start it holds k * gridDim.x (k calls done), every block adds one,
 // and all wait until it reaches (k + 1) * gridDim.x, with a bounded number of
-// polls.  Both are called by every thread of the block.
+// polls (the handle's limit; a test hook can also add arrivals that never
+// come, so every block gives up while the counter stays a multiple of the
+// grid).  Both are called by every thread of the block.
 __device__ void grid_arrive(unsigned long long *ctr) {
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -144,13 +146,13 @@ __device__ void grid_arrive(unsigned long long *ctr) {
     }
 }
 
-__device__ bool grid_wait(unsigned long long *ctr, unsigned long long target) {
+__device__ bool grid_wait(unsigned long long *ctr, unsigned long long target, uint32_t polls) {
     __shared__ int s_ok;
     __syncthreads();
     if (threadIdx.x == 0) {
         int ok = 0;
         const volatile unsigned long long *v = ctr;
-        for (uint32_t it = 0; it < kBarrierPolls; ++it) {
+        for (uint32_t it = 0; it < polls; ++it) {
             if (*v >= target) {
                 ok = 1;
                 break;
@@ -435,15 +437,10 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
         const int e = ent_e[i];
         if (e != 0xFFFF) ent_rank[i] = (uint16_t)(ent_rank[i] + wcnt[(i >> lg_run) * E + e]);
     }
-    PLAN_TRACE(5);
-    if (!grid_wait(a.ws.arrive, (call + 1) * gridDim.x)) {
-        if (tid == 0) atomicOr(a.plan.status, MOONEP_STATUS_TIMEOUT);
-        return;
-    }
-    PLAN_TRACE(1);
-    // the next call's error slot: every block of this call is past its last
-    // write to the other slot's counterpart, and the next call starts after
-    // this kernel ends
+    // The next call's tables (the other parity) start at zero.  No block of
+    // this call reads or writes them, and the next call starts after this
+    // kernel ends, so they are cleared here, before the wait: a block that
+    // gives up waiting still leaves them clean.
     if (blockIdx.x == 0 && tid == 0) a.ws.status[parity ^ 1] = 0;
     if (blockIdx.x == 0 && tid < R) a.ws.gload[(size_t)(parity ^ 1) * R + tid] = 0;
     {
@@ -453,6 +450,12 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
              i += kPlanThreads)
             next[i] = 0;
     }
+    PLAN_TRACE(5);
+    if (!grid_wait(a.ws.arrive, (call + 1) * gridDim.x + a.withheld, a.polls)) {
+        if (tid == 0) atomicOr(a.plan.status, MOONEP_STATUS_TIMEOUT);
+        return;
+    }
+    PLAN_TRACE(1);
 
     // ---------------- B. layout (every block) ----------------
     // T and pre are rewritten, once the outputs no longer need them, into the

@@ -121,3 +121,67 @@ def test_host_side_errors(cuda):
         moonep.moonep_prefetch_weight(h, p, [W] * 9, [pool] * 9)
     assert e.value.code == moonep.ERR_SIZE
     h.close()
+
+
+def test_planner_barrier_timeout_is_reported_and_the_handle_recovers(cuda):
+    # A bounded wait made to run out from the host: the hook makes the
+    # planner's grid barrier wait for one block arrival that never comes and
+    # give up after a few thousand polls.  Every block returns with
+    # MOONEP_STATUS_TIMEOUT within milliseconds, and the tables the next call
+    # uses are left clean, so the same handle plans bit-exactly afterwards
+    # (the timed-out call is not the handle's first, so its count tables were
+    # in use).  A fresh handle plans bit-exactly too.
+    import time
+
+    from load_balancing_planner_b200 import moonep
+    Rz, Sz, Kz, Ez, Bz, tp = 8, 1024, 8, 64, 8, 128
+    tk, tpe, _ = problem(Rz, Sz, Kz, Ez, 2.0, "zipf", seed=3)
+    tk2, tpe2, _ = problem(Rz, Sz, Kz, Ez, 0.5, "zipf", seed=4)
+    h = moonep.moonep_create(Sz, 8, Kz, Ez, Rz, Bz, tp)
+    warm = plan_to_numpy(gpu_plan(h, tk2, tpe2))
+    assert_plans_equal(warm, oracle.plan(tk2, Ez, Bz, tp, 0, tpe2))
+
+    moonep.moonep_set_plan_barrier(h, 4096, 1)
+    p = moonep.Plan(h)
+    p.dst.fill_(-7)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    moonep.moonep_plan(h, torch.from_numpy(tk).cuda(), torch.from_numpy(tpe).cuda(), p)
+    st = moonep.moonep_read_status(p)
+    dt = time.perf_counter() - t0
+    assert st == moonep.STATUS_TIMEOUT
+    assert dt < 1.0, dt
+    assert bool((p.dst == -7).all())  # nothing past the barrier was written
+    assert moonep.moonep_plan_status(p) == moonep.STATUS_TIMEOUT
+    # later calls on the timed-out plan do nothing
+    x = synth.hidden_bf16(Rz, Sz, 8, seed=1).cuda()
+    buf = torch.empty((Rz, h.nvs, 8), dtype=torch.int16, device="cuda").fill_(-1).view(torch.bfloat16)
+    moonep.moonep_dispatch(h, p, x, None, buf)
+    torch.cuda.synchronize()
+    assert bool((buf.view(torch.int16) == -1).all())
+
+    moonep.moonep_set_plan_barrier(h, 0, 0)
+    want = oracle.plan(tk, Ez, Bz, tp, 0, tpe)
+    for _ in range(2):  # both parities of the handle's tables
+        assert_plans_equal(plan_to_numpy(gpu_plan(h, tk, tpe)), want)
+
+    # the one-rank planner of the same handle: its own barrier, same hook
+    c = torch.from_numpy(tpe).cuda()
+    moonep.moonep_set_plan_barrier(h, 4096, 2)
+    pr = moonep.moonep_plan_rank(h, 3, torch.from_numpy(np.ascontiguousarray(tk[3])).cuda(), c)
+    assert moonep.moonep_read_status(pr) == moonep.STATUS_TIMEOUT
+    moonep.moonep_set_plan_barrier(h, 0, 0)
+    wr = oracle.plan_rank(tk[3], tpe, 3, Ez, Bz, tp, 0)
+    for _ in range(2):
+        pr = moonep.moonep_plan_rank(h, 3, torch.from_numpy(np.ascontiguousarray(tk[3])).cuda(), c)
+        assert moonep.moonep_read_status(pr) == 0
+        assert np.array_equal(pr.dst.cpu().numpy(), wr["dst"])
+        assert np.array_equal(pr.cu_seqlens.cpu().numpy(), wr["cu_seqlens"])
+    h.close()
+
+    fresh = moonep.moonep_create(Sz, 8, Kz, Ez, Rz, Bz, tp)
+    assert_plans_equal(plan_to_numpy(gpu_plan(fresh, tk, tpe)), want)
+    with pytest.raises(moonep.MoonepError) as e:
+        moonep.moonep_set_plan_barrier(fresh, 0, -1)
+    assert e.value.code == moonep.ERR_SIZE
+    fresh.close()
