@@ -20,7 +20,8 @@
  *    owns every tensor, including the plan arrays; the library owns only the
  *    handle and a small planning workspace inside it.
  *  - Every call is asynchronous on `stream` (NULL = legacy default stream) and
- *    never synchronises the host, except moonep_read_status.
+ *    never synchronises the host, except moonep_read_status and
+ *    moonep_plan_status.
  *  - Return value: MOONEP_OK, or a negative MOONEP_ERR_* for errors detected
  *    on the host before anything is launched.  Data-dependent errors are found
  *    on the device and reported as MOONEP_STATUS_* bits in plan->status; every
@@ -63,7 +64,7 @@ typedef struct CUstream_st *moonep_stream_t;
 #define MOONEP_STATUS_DUP_EXPERT 2     /* an expert picked twice by one token */
 #define MOONEP_STATUS_COUNT_MISMATCH 4 /* tokens_per_expert differs from the picks */
 #define MOONEP_STATUS_BAD_PLAN 8       /* a plan index pointed outside its buffer; skipped */
-#define MOONEP_STATUS_TIMEOUT 16       /* the planner's grid barrier gave up waiting; destroy the handle */
+#define MOONEP_STATUS_TIMEOUT 16       /* the planner's grid barrier gave up waiting (see moonep_set_plan_barrier) */
 
 /* Supported ranges (moonep_create checks them). */
 #define MOONEP_MAX_R 64
@@ -120,6 +121,28 @@ typedef struct {
 } moonep_plan_t;
 
 typedef struct moonep_handle *moonep_handle_t;
+
+/*
+ * Element counts of the plan arrays for a configuration, so that a caller can
+ * allocate a moonep_plan_t before any handle exists (the README's
+ * "MoonEPCommPlan", "dispatch fwd", is kept by the caller for the later
+ * calls).  Every count is in elements of the array's own type:
+ *   dst          R*S*K (group plan) or S*K (one rank's plan, one_rank != 0)
+ *   cu_seqlens   R*(E+B)            row_counts  R*(E+B)
+ *   slot_expert  R*B (0 when B = 0; the pointer may then be NULL)
+ *   counts       R*E                assign      R*4
+ *   maxvio       1 float            status      1 int32
+ *   nvs          NvS, the slots of one rank's dispatch buffer (moonep_nvs):
+ *                hidden_nvs holds R*NvS rows of H bf16, route_weights_nvs
+ *                R*NvS floats (one rank's buffers: NvS each)
+ * Host only: no device is touched.  Returns MOONEP_ERR_NULL for a NULL
+ * argument, or cfg's moonep_create error (MOONEP_ERR_CONFIG) with *out
+ * zeroed.
+ */
+typedef struct {
+    int64_t dst, cu_seqlens, row_counts, slot_expert, counts, assign, maxvio, status, nvs;
+} moonep_plan_sizes_t;
+MOONEP_API int moonep_plan_sizes(const moonep_config_t *cfg, int32_t one_rank, moonep_plan_sizes_t *out);
 
 /*
  * Validate cfg and create a handle on the current device; allocates the
@@ -353,8 +376,11 @@ MOONEP_API int moonep_reduce_grad_rank(moonep_handle_t h, const moonep_plan_t *p
  * start at zero with cudaMemsetAsync on `stream`.
  *
  * The first call on a device looks the array's device address up
- * (cudaGetSymbolAddress, with that device current); make that first call
- * before any stream capture.  All calls share the one array: calls that
+ * (cudaGetSymbolAddress, with that device current) and keeps it for the
+ * life of the process; make that first call before any stream capture, and
+ * do not use the library across a cudaDeviceReset (the kept address, like
+ * the kernel attributes every entry point sets once per device, would be
+ * stale).  All calls share the one array: calls that
  * overlap on the GPU race, so order them on one stream.  Arguments, layouts
  * and status bits are those of moonep_plan; cfg is checked as moonep_create
  * checks it.
@@ -364,8 +390,28 @@ MOONEP_API int moonep_plan_noalloc(const moonep_config_t *cfg, const int32_t *to
                                    const int32_t *tokens_per_expert, const moonep_plan_t *plan,
                                    moonep_stream_t stream);
 
-/* Read plan->status into *status (host).  Synchronises `stream`. */
+/* Read plan->status into *status (host).  Synchronises `stream`.  This is
+ * the status read of the library's scope (named moonep_plan_status there),
+ * with the stream made explicit; moonep_plan_status below is the stream-less
+ * form. */
 MOONEP_API int moonep_read_status(const moonep_plan_t *plan, int32_t *status, moonep_stream_t stream);
+
+/* Read plan->status into *status after waiting for all work on the current
+ * device (cudaDeviceSynchronize), whatever stream wrote it. */
+MOONEP_API int moonep_plan_status(const moonep_plan_t *plan, int32_t *status);
+
+/*
+ * Fault injection for tests, on the host side (nothing faults on the GPU).
+ * The planner's grid barrier of handle h (moonep_plan and moonep_plan_rank)
+ * gives up after max_polls polls (0 restores the default, about 2 s of
+ * polling) and, with missing > 0, also waits for `missing` block arrivals
+ * that never come, so that every block gives up.  The call then sets
+ * MOONEP_STATUS_TIMEOUT in plan->status and writes no other plan array;
+ * later calls on the plan do nothing.  A timeout caused this way leaves the
+ * handle usable: restore (0, 0) and plan again.  After a timeout of any other
+ * cause, destroy the handle.  ERR_SIZE when missing is outside [0, 2^20].
+ */
+MOONEP_API int moonep_set_plan_barrier(moonep_handle_t h, uint32_t max_polls, int32_t missing);
 
 /* Static description of a MOONEP_ERR_* code. */
 MOONEP_API const char *moonep_error_string(int code);

@@ -28,6 +28,8 @@ struct moonep_handle {
     void *ws_mem;
     Workspace ws;
     Workspace ws_rank;  // one-rank planning (moonep_plan_rank): its own barrier counter and parity slots
+    uint32_t barrier_polls;     // the planner's grid-barrier poll limit
+    uint32_t barrier_withheld;  // arrivals that never come (fault injection for tests; normally 0)
 };
 
 // Handle workspace: [group planning][group GEMM pair table][one-rank planning]
@@ -185,6 +187,8 @@ extern "C" int moonep_create(const moonep_config_t *cfg, moonep_handle_t *out) {
     }
     carve_workspace(d, h->ws_mem, &h->ws);
     carve_workspace(d, static_cast<char *>(h->ws_mem) + rank_ws_offset(d), &h->ws_rank);
+    h->barrier_polls = kBarrierPolls;
+    h->barrier_withheld = 0;
     *out = h;
     return MOONEP_OK;
 }
@@ -195,6 +199,14 @@ extern "C" int moonep_destroy(moonep_handle_t h) {
     if (h->ws_mem) e = cudaFree(h->ws_mem);
     free(h);
     return e == cudaSuccess ? MOONEP_OK : MOONEP_ERR_CUDA;
+}
+
+extern "C" int moonep_set_plan_barrier(moonep_handle_t h, uint32_t max_polls, int32_t missing) {
+    if (!h) return MOONEP_ERR_NULL;
+    if (missing < 0 || missing > (1 << 20)) return MOONEP_ERR_SIZE;
+    h->barrier_polls = max_polls ? max_polls : kBarrierPolls;
+    h->barrier_withheld = (uint32_t)missing;
+    return MOONEP_OK;
 }
 
 extern "C" int64_t moonep_nvs(moonep_handle_t h) { return h ? (int64_t)h->d.nvs : MOONEP_ERR_NULL; }
@@ -217,6 +229,8 @@ extern "C" int moonep_plan(moonep_handle_t h, const int32_t *topk, const int32_t
     a.counts_all = nullptr;
     a.plan = *plan;
     a.ws = h->ws;
+    a.polls = h->barrier_polls;
+    a.withheld = h->barrier_withheld;
     const cudaError_t e = launch_plan(a, h->grid_plan, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? MOONEP_OK : fail_cuda(e);
 }
@@ -234,6 +248,8 @@ extern "C" int moonep_plan_rank(moonep_handle_t h, int32_t rank, const int32_t *
     a.counts_all = counts_all;
     a.plan = *plan;
     a.ws = h->ws_rank;
+    a.polls = h->barrier_polls;
+    a.withheld = h->barrier_withheld;
     const cudaError_t e = launch_plan(a, h->d.nch, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? MOONEP_OK : fail_cuda(e);
 }
@@ -434,6 +450,31 @@ extern "C" int moonep_group_gemm(moonep_handle_t h, const moonep_plan_t *plan, c
     if (rc != MOONEP_OK) return rc;
     int32_t *pairs = reinterpret_cast<int32_t *>(static_cast<char *>(h->ws_mem) + pair_table_offset(h->d));
     return launch_group_gemm(h->d, plan, x_nvs, weights, pool, y_nvs, Hp, pairs, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int moonep_plan_sizes(const moonep_config_t *cfg, int32_t one_rank, moonep_plan_sizes_t *out) {
+    if (!cfg || !out) return MOONEP_ERR_NULL;
+    memset(out, 0, sizeof(*out));
+    const int rc = check_config(*cfg);
+    if (rc != MOONEP_OK) return rc;
+    const int64_t R = cfg->R, S = cfg->S, K = cfg->K, E = cfg->E, B = cfg->B;
+    out->dst = one_rank ? S * K : R * S * K;
+    out->cu_seqlens = R * (E + B);
+    out->row_counts = R * (E + B);
+    out->slot_expert = R * B;
+    out->counts = R * E;
+    out->assign = R * 4;
+    out->maxvio = 1;
+    out->status = 1;
+    out->nvs = nvs_of(*cfg);
+    return MOONEP_OK;
+}
+
+extern "C" int moonep_plan_status(const moonep_plan_t *plan, int32_t *status) {
+    if (!plan || !plan->status || !status) return MOONEP_ERR_NULL;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e == cudaSuccess) e = cudaMemcpy(status, plan->status, sizeof(int32_t), cudaMemcpyDeviceToHost);
+    return e == cudaSuccess ? MOONEP_OK : fail_cuda(e);
 }
 
 extern "C" int moonep_read_status(const moonep_plan_t *plan, int32_t *status, moonep_stream_t stream) {

@@ -34,6 +34,11 @@ class Config(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("S", "H", "K", "E", "R", "B", "token_padding", "num_sms", "mode")]
 
 
+class PlanSizes(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in
+                ("dst", "cu_seqlens", "row_counts", "slot_expert", "counts", "assign", "maxvio", "status", "nvs")]
+
+
 class PlanStruct(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("dst", "cu_seqlens", "row_counts", "slot_expert", "counts", "assign", "maxvio", "status")]
@@ -56,6 +61,9 @@ def _load():
         "moonep_prefetch_weight": ([P, ctypes.POINTER(PlanStruct), i32, P, P, i64, P], ctypes.c_int),
         "moonep_reduce_grad": ([P, ctypes.POINTER(PlanStruct), i32, P, P, i64, P], ctypes.c_int),
         "moonep_read_status": ([ctypes.POINTER(PlanStruct), ctypes.POINTER(i32), P], ctypes.c_int),
+        "moonep_plan_status": ([ctypes.POINTER(PlanStruct), ctypes.POINTER(i32)], ctypes.c_int),
+        "moonep_plan_sizes": ([ctypes.POINTER(Config), i32, ctypes.POINTER(PlanSizes)], ctypes.c_int),
+        "moonep_set_plan_barrier": ([P, ctypes.c_uint32, i32], ctypes.c_int),
         "moonep_error_string": ([ctypes.c_int], ctypes.c_char_p),
         "moonep_last_error": ([], ctypes.c_char_p),
         "moonep_plan_noalloc": ([ctypes.POINTER(Config), P, P, ctypes.POINTER(PlanStruct), P], ctypes.c_int),
@@ -78,7 +86,8 @@ EXPORTS = ("moonep_create", "moonep_destroy", "moonep_nvs", "moonep_get_config",
            "moonep_dispatch", "moonep_combine", "moonep_prefetch_weight", "moonep_reduce_grad",
            "moonep_read_status", "moonep_error_string", "moonep_last_error", "moonep_plan_noalloc",
            "moonep_group_gemm", "moonep_plan_rank", "moonep_dispatch_rank", "moonep_combine_rank",
-           "moonep_prefetch_weight_rank", "moonep_reduce_grad_rank")
+           "moonep_prefetch_weight_rank", "moonep_reduce_grad_rank", "moonep_plan_sizes", "moonep_plan_status",
+           "moonep_set_plan_barrier")
 NOALLOC_SCRATCH_BYTES = 1 << 20
 
 
@@ -146,16 +155,19 @@ class Plan:
     def __init__(self, h, device=None, rank: int | None = None):
         dev = device or torch.device("cuda", torch.cuda.current_device())
         R, S, K, E, B = h.R, h.S, h.K, h.E, h.B
+        # element counts from the C ABI (moonep_plan_sizes), viewed in the
+        # arrays' documented shapes
+        sz = moonep_plan_sizes(h.cfg if isinstance(h, Handle) else h, rank is not None)
         i32 = dict(dtype=torch.int32, device=dev)
         self.rank = rank
-        self.dst = torch.empty((S, K) if rank is not None else (R, S, K), **i32)
-        self.cu_seqlens = torch.empty((R, E + B), **i32)
-        self.row_counts = torch.empty((R, E + B), **i32)
-        self.slot_expert = torch.empty((R, max(B, 1)), **i32)
-        self.counts = torch.empty((R, E), **i32)
-        self.assign = torch.empty((R, 4), **i32)
-        self.maxvio = torch.empty((1,), dtype=torch.float32, device=dev)
-        self.status = torch.zeros((1,), **i32)
+        self.dst = torch.empty(sz.dst, **i32).view((S, K) if rank is not None else (R, S, K))
+        self.cu_seqlens = torch.empty(sz.cu_seqlens, **i32).view(R, E + B)
+        self.row_counts = torch.empty(sz.row_counts, **i32).view(R, E + B)
+        self.slot_expert = torch.empty(max(sz.slot_expert, R), **i32).view(R, max(B, 1))
+        self.counts = torch.empty(sz.counts, **i32).view(R, E)
+        self.assign = torch.empty(sz.assign, **i32).view(R, 4)
+        self.maxvio = torch.empty(sz.maxvio, dtype=torch.float32, device=dev)
+        self.status = torch.zeros(sz.status, **i32)
         self.struct = PlanStruct(*(t.data_ptr() for t in (
             self.dst, self.cu_seqlens, self.row_counts, self.slot_expert, self.counts,
             self.assign, self.maxvio, self.status)))
@@ -164,6 +176,19 @@ class Plan:
 
     def slots(self):
         return self.slot_expert[:, : self.B]
+
+
+def moonep_plan_sizes(cfg: Config, one_rank: bool = False) -> PlanSizes:
+    """Element counts of the plan arrays for cfg (and NvS), from the C ABI."""
+    out = PlanSizes()
+    _check(lib.moonep_plan_sizes(ctypes.byref(cfg), 1 if one_rank else 0, ctypes.byref(out)), "moonep_plan_sizes")
+    return out
+
+
+def moonep_set_plan_barrier(h: "Handle", max_polls: int = 0, missing: int = 0):
+    """Test hook: the planner's grid barrier of h gives up after max_polls
+    polls and waits for `missing` arrivals that never come ((0, 0) = normal)."""
+    _check(lib.moonep_set_plan_barrier(h.ptr, max_polls, missing), "moonep_set_plan_barrier")
 
 
 def moonep_create(S, H, K, E, R, B=None, token_padding=128, num_sms=0, mode=TRAINING) -> Handle:
@@ -406,6 +431,13 @@ def moonep_group_gemm(h: Handle, plan: Plan, x_nvs, weights, pool=None, y_nvs=No
     _check(lib.moonep_group_gemm(h.ptr, ctypes.byref(plan.struct), _ptr(x_nvs), _ptr(weights), _ptr(pool),
                                  _ptr(y_nvs), Hp, _stream(stream)), "moonep_group_gemm")
     return y_nvs
+
+
+def moonep_plan_status(plan: Plan) -> int:
+    """plan.status after waiting for all work on the current device."""
+    st = ctypes.c_int32(0)
+    _check(lib.moonep_plan_status(ctypes.byref(plan.struct), ctypes.byref(st)), "moonep_plan_status")
+    return int(st.value)
 
 
 def moonep_read_status(plan: Plan, stream=None) -> int:

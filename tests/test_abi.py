@@ -126,12 +126,17 @@ C_CALLER = r"""
 #include "moonep.h"
 int main(void) {
     moonep_config_t c = {64, 128, 2, 10, 4, 4, 8, 0, 0};  /* E % R != 0 */
+    moonep_config_t ok = {64, 128, 2, 8, 2, 4, 8, 0, 0};
     moonep_handle_t h = (moonep_handle_t)0;
+    moonep_plan_sizes_t sz;
     if (moonep_create(&c, &h) != MOONEP_ERR_CONFIG || h) return 1;
     if (strcmp(moonep_error_string(MOONEP_ERR_CONFIG), "configuration rejected") != 0) return 2;
     if (moonep_plan_rank(0, 0, 0, 0, 0, 0) != MOONEP_ERR_NULL) return 3;
     if (moonep_dispatch_rank(0, 0, 0, 0, 0, 0, 0) != MOONEP_ERR_NULL) return 4;
     if (moonep_destroy(0) != MOONEP_OK) return 5;
+    if (moonep_plan_sizes(&c, 0, &sz) != MOONEP_ERR_CONFIG || sz.dst != 0) return 6;
+    if (moonep_plan_sizes(&ok, 0, &sz) != MOONEP_OK || sz.dst != 2 * 64 * 2 || sz.nvs != 184) return 7;
+    if (moonep_plan_status(0, 0) != MOONEP_ERR_NULL || moonep_set_plan_barrier(0, 0, 0) != MOONEP_ERR_NULL) return 8;
     puts("ok");
     return 0;
 }
@@ -153,3 +158,170 @@ def test_header_is_plain_c_and_the_library_links_from_c(tmp_path):
                     f"-Wl,-rpath,{libdir}"], check=True)
     out = subprocess.run([str(exe)], capture_output=True, text=True)
     assert out.returncode == 0 and out.stdout.strip() == "ok", (out.returncode, out.stdout, out.stderr)
+
+
+@pytest.mark.parametrize("R,S,K,E,B,tp,mode", [(2, 64, 2, 8, 4, 8, 0), (8, 4096, 8, 256, 32, 128, 0),
+                                               (8, 4096, 8, 256, 4, 128, 1), (4, 333, 3, 24, 0, 16, 1),
+                                               (64, 40, 4, 256, 4, 8, 2)])
+def test_plan_sizes_match_the_oracle_arrays(R, S, K, E, B, tp, mode):
+    # moonep_plan_sizes (host only) against the shapes of the arrays the
+    # oracle fills for the same configuration, group and one-rank forms
+    import numpy as np
+
+    import oracle
+    from load_balancing_planner_b200 import moonep
+    cfg = moonep.Config(S, 8, K, E, R, B, tp, 0, mode)
+    sz = moonep.moonep_plan_sizes(cfg)
+    rng = np.random.default_rng(0)
+    tk = np.stack([np.stack([rng.permutation(E)[:K] for _ in range(S)]) for _ in range(R)]).astype(np.int32)
+    o = oracle.plan(tk, E, B, tp, mode)
+    assert o["status"] == 0
+    for k in ("dst", "cu_seqlens", "row_counts", "slot_expert", "counts", "assign"):
+        assert getattr(sz, k) == o[k].size, k
+    assert sz.maxvio == 1 and sz.status == 1
+    assert sz.nvs == o["nvs"] == oracle.nvs(S, K, E, R, tp)
+    counts = np.stack([np.bincount(tk[r].reshape(-1), minlength=E) for r in range(R)]).astype(np.int32)
+    orank = oracle.plan_rank(tk[R - 1], counts, R - 1, E, B, tp, mode)
+    assert moonep.moonep_plan_sizes(cfg, True).dst == orank["dst"].size == S * K
+
+
+C_GPU_CALLER = r"""
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+#include <cuda_runtime_api.h>
+#include "moonep.h"
+
+/* Plans and dispatches one layer through the C ABI, with every device array
+   sized from moonep_plan_sizes alone.  argv: input file (topk int32 [R*S*K],
+   tokens_per_expert int32 [R*E], hidden bf16 bits [R*S*H], route weights fp32
+   [R*S*K]), output file (the plan arrays in moonep_plan_t order, then the
+   dispatch buffer [R*NvS*H] and its weights [R*NvS]). */
+static void *dev(int64_t bytes, unsigned char fill) {
+    void *p = NULL;
+    if (cudaMalloc(&p, (size_t)(bytes > 0 ? bytes : 4)) != cudaSuccess) exit(20);
+    if (cudaMemset(p, fill, (size_t)(bytes > 0 ? bytes : 4)) != cudaSuccess) exit(21);
+    return p;
+}
+static void *up(FILE *f, int64_t bytes) {
+    void *h = malloc((size_t)bytes), *d = dev(bytes, 0);
+    if (!h || fread(h, 1, (size_t)bytes, f) != (size_t)bytes) exit(22);
+    if (cudaMemcpy(d, h, (size_t)bytes, cudaMemcpyHostToDevice) != cudaSuccess) exit(23);
+    free(h);
+    return d;
+}
+static void down(FILE *f, const void *d, int64_t bytes) {
+    void *h = malloc((size_t)bytes);
+    if (!h || cudaMemcpy(h, d, (size_t)bytes, cudaMemcpyDeviceToHost) != cudaSuccess) exit(24);
+    if (fwrite(h, 1, (size_t)bytes, f) != (size_t)bytes) exit(25);
+    free(h);
+}
+int main(int argc, char **argv) {
+    moonep_config_t c = {64, 128, 2, 8, 2, 4, 8, 0, 0};
+    moonep_plan_sizes_t n;
+    moonep_plan_t p;
+    moonep_handle_t h = NULL;
+    int32_t st = -1;
+    FILE *in, *out;
+    void *topk, *tpe, *hidden, *w, *buf, *wbuf;
+    const int64_t R = c.R, S = c.S, K = c.K, E = c.E, H = c.H;
+    if (argc != 3 || !(in = fopen(argv[1], "rb")) || !(out = fopen(argv[2], "wb"))) return 10;
+    if (moonep_plan_sizes(&c, 0, &n) != MOONEP_OK) return 11;
+    p.dst = (int32_t *)dev(4 * n.dst, 0xFF);
+    p.cu_seqlens = (int32_t *)dev(4 * n.cu_seqlens, 0xFF);
+    p.row_counts = (int32_t *)dev(4 * n.row_counts, 0xFF);
+    p.slot_expert = (int32_t *)dev(4 * n.slot_expert, 0xFF);
+    p.counts = (int32_t *)dev(4 * n.counts, 0xFF);
+    p.assign = (int32_t *)dev(4 * n.assign, 0xFF);
+    p.maxvio = (float *)dev(4 * n.maxvio, 0xFF);
+    p.status = (int32_t *)dev(4 * n.status, 0xFF);
+    topk = up(in, 4 * R * S * K);
+    tpe = up(in, 4 * R * E);
+    hidden = up(in, 2 * R * S * H);
+    w = up(in, 4 * R * S * K);
+    buf = dev(2 * R * n.nvs * H, 0xFF);
+    wbuf = dev(4 * R * n.nvs, 0xFF);
+    if (moonep_create(&c, &h) != MOONEP_OK) return 12;
+    if (moonep_nvs(h) != n.nvs) return 13;
+    if (moonep_plan(h, (const int32_t *)topk, (const int32_t *)tpe, &p, NULL) != MOONEP_OK) return 14;
+    if (moonep_dispatch(h, &p, hidden, (const float *)w, buf, (float *)wbuf, NULL) != MOONEP_OK) return 15;
+    if (moonep_plan_status(&p, &st) != MOONEP_OK || st != 0) return 16;
+    down(out, p.dst, 4 * n.dst);
+    down(out, p.cu_seqlens, 4 * n.cu_seqlens);
+    down(out, p.row_counts, 4 * n.row_counts);
+    down(out, p.slot_expert, 4 * n.slot_expert);
+    down(out, p.counts, 4 * n.counts);
+    down(out, p.assign, 4 * n.assign);
+    down(out, p.maxvio, 4 * n.maxvio);
+    down(out, p.status, 4 * n.status);
+    down(out, buf, 2 * R * n.nvs * H);
+    down(out, wbuf, 4 * R * n.nvs);
+    fclose(out);
+    fclose(in);
+    if (moonep_destroy(h) != MOONEP_OK) return 17;
+    puts("ok");
+    return 0;
+}
+"""
+
+
+@pytest.mark.gpu
+def test_c_caller_sizes_plans_and_dispatches_on_the_gpu(tmp_path, cuda):
+    # a C99 program allocates a plan from moonep_plan_sizes alone, plans and
+    # dispatches the tiny case on the GPU; its plan is bit-exact against the
+    # oracle and so is the dispatch buffer, untouched padding included
+    import subprocess
+
+    import numpy as np
+
+    import oracle
+    from load_balancing_planner_b200 import build, synth
+    R, S, K, E, B, H, tp = 2, 64, 2, 8, 4, 128, 8
+    tk, _, _ = synth.routing(R, S, K, E, 1.0, "boost0", seed=0)
+    tpe = synth.local_counts(tk, E)
+    xb = synth.bf16_bits(synth.hidden_bf16(R, S, H, seed=0))
+    w = synth.route_weights(R, S, K, seed=0)
+    inp = tmp_path / "in.bin"
+    with open(inp, "wb") as f:
+        for a in (tk.astype(np.int32), tpe.astype(np.int32), xb.astype(np.uint16), w.astype(np.float32)):
+            f.write(np.ascontiguousarray(a).tobytes())
+    lib = build.build()
+    src = tmp_path / "gpu_caller.c"
+    src.write_text(C_GPU_CALLER)
+    exe = tmp_path / "gpu_caller"
+    libdir = os.path.dirname(lib)
+    cuda_home = os.environ.get("CUDA_HOME", "/usr/local/cuda")
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    "-I", os.path.join(cuda_home, "include"), "-o", str(exe), str(src), "-L", libdir, "-lmoonep",
+                    "-L", os.path.join(cuda_home, "lib64"), "-lcudart",
+                    f"-Wl,-rpath,{libdir}", f"-Wl,-rpath,{os.path.join(cuda_home, 'lib64')}"], check=True)
+    outp = tmp_path / "out.bin"
+    r = subprocess.run([str(exe), str(inp), str(outp)], capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stdout, r.stderr)
+
+    o = oracle.plan(tk, E, B, tp, 0, tpe)
+    nvs = o["nvs"]
+    raw = open(outp, "rb").read()
+    off = 0
+
+    def take(dtype, n):
+        nonlocal off
+        a = np.frombuffer(raw, dtype=dtype, count=n, offset=off)
+        off += a.nbytes
+        return a
+
+    got = {}
+    for k in ("dst", "cu_seqlens", "row_counts", "slot_expert", "counts", "assign"):
+        got[k] = take(np.int32, o[k].size).reshape(o[k].shape)
+        assert np.array_equal(got[k], o[k]), k
+    assert np.float32(take(np.float32, 1)[0]) == np.float32(o["maxvio"])
+    assert take(np.int32, 1)[0] == 0
+    gbuf = take(np.uint16, R * nvs * H).reshape(R * nvs, H)
+    gw = take(np.uint32, R * nvs)
+    assert off == len(raw)
+    obuf, own = oracle.dispatch(o["dst"], xb, w, nvs)
+    assert np.array_equal(gbuf, obuf)  # real slots and the untouched 0xFFFF padding
+    live = o["dst"].reshape(-1)
+    assert np.array_equal(gw[live], own[live].view(np.uint32))
+    dead = np.setdiff1d(np.arange(R * nvs), live)
+    assert np.all(gw[dead] == 0xFFFFFFFF)
