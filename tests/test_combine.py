@@ -105,3 +105,41 @@ def test_combine_training_shape_sampled(cuda):
     assert ok.all()
     assert np.array_equal(gw.view(R * S, K)[torch.from_numpy(toks).cuda()].cpu().numpy(), ogw[0])
     h.close()
+
+
+def test_dispatch_combine_inference_shape_sampled(cuda):
+    # the inference shape (R=8, S=4096, K=8, E=256, B=4, H=7168, maxvio 4):
+    # copies past the B slots are read from their home rows.  Dispatch then a
+    # weighted combine of the dispatched buffer; 512 tokens against the
+    # oracle's dispatch and combine of those tokens' picks, one by one
+    from load_balancing_planner_b200 import moonep
+    R, S, K, E, B, H, tp = 8, 4096, 8, 256, 4, 7168, 128
+    tk, tpe, _ = problem(R, S, K, E, 4.0, "hot8", seed=12)
+    xh = synth.hidden_bf16(R, S, H, seed=12)
+    wh = synth.route_weights(R, S, K, seed=12)
+    h = moonep.moonep_create(S, H, K, E, R, B, tp, mode=1)
+    p = gpu_plan(h, tk, tpe)
+    o = oracle.plan(tk, E, B, tp, 1, tpe)
+    assert np.array_equal(p.dst.cpu().numpy(), o["dst"])
+    home = np.arange(E) // (E // R)
+    assert any(o["row_counts"][r, e] > 0 for r in range(R) for e in range(E) if home[e] != r), "no overflow rows"
+    buf, wn = moonep.moonep_dispatch(h, p, xh.cuda(), torch.from_numpy(wh).cuda())
+    out, gw = moonep.moonep_combine(h, p, buf, wn)
+    torch.cuda.synchronize()
+    assert moonep.moonep_read_status(p) == 0
+    rng = np.random.default_rng(12)
+    toks = rng.choice(R * S, size=512, replace=False)
+    d = o["dst"].reshape(R * S, K)[toks]                        # [n, K] slots of the sampled picks
+    dsmall = np.arange(len(toks) * K, dtype=np.int32).reshape(1, len(toks), K)
+    xb = synth.bf16_bits(xh).reshape(R * S, H)[toks].reshape(1, len(toks), H)
+    wsm = wh.reshape(R * S, K)[toks].reshape(1, len(toks), K)
+    obuf, own = oracle.dispatch(dsmall, xb, wsm, len(toks) * K)  # the oracle's slots, renumbered
+    sl = torch.from_numpy(d.reshape(-1)).cuda().long()
+    assert np.array_equal(bits(buf.view(-1, H)[sl]), obuf)
+    assert np.array_equal(wn.view(-1)[sl].cpu().numpy().view(np.uint32), own.view(np.uint32))
+    oout, ogw = oracle.combine(dsmall, obuf, own)
+    g = bf16_to_f64(bits(out.view(R * S, H)[torch.from_numpy(toks).cuda()]))
+    ok = rel_close(g, bf16_to_f64(oout[0]), RTOL_BF16)
+    assert ok.all(), f"{(~ok).sum()} of {ok.size} outside tolerance"
+    assert np.array_equal(gw.view(R * S, K)[torch.from_numpy(toks).cuda()].cpu().numpy(), ogw[0])
+    h.close()

@@ -43,29 +43,64 @@ def test_dispatch_matches_oracle(cuda, R, S, K, E, B, H, tp, mode, profile, mv):
     h.close()
 
 
-def test_dispatch_training_shape_full(cuda):
-    # R=8, S=4096, K=8, E=256, B=32, H=7168 at maxvio 2: every (token, k) row
-    # is checked through the plan on the device, padding rows stay sentinel
+def _sampled_oracle_rows(o, xb, w, toks):
+    """The oracle's own dispatch of the picks of tokens `toks` (same ids on
+    every source rank): its slots renumbered compactly in slot order, so the
+    oracle writes a small buffer.  Returns (the plan's slots of those picks,
+    flat [n]; the oracle's rows for them [n, H]; their weights [n])."""
+    dsub = np.ascontiguousarray(o["dst"][:, toks, :])         # [R, n_tok, K]
+    flat = dsub.reshape(-1)
+    order = np.argsort(flat, kind="stable")
+    comp = np.empty(flat.size, np.int32)
+    comp[order] = np.arange(flat.size, dtype=np.int32)
+    R = dsub.shape[0]
+    obuf, own = oracle.dispatch(comp.reshape(dsub.shape), np.ascontiguousarray(xb[:, toks, :]),
+                                np.ascontiguousarray(w[:, toks, :]), flat.size // R)
+    return flat, obuf[comp], own[comp]
+
+
+@pytest.mark.parametrize("B,mode,mv", [(32, 0, 2.0), (4, 1, 4.0)], ids=["train_mv2", "infer_mv4"])
+def test_dispatch_full_shape_sampled_against_oracle(cuda, B, mode, mv):
+    # R=8, S=4096, K=8, E=256, H=7168 at the training shape (B=32) and the
+    # inference shape (B=4, copies past B read from their home rows): the
+    # plan is bit-exact; the rows and weights of 256 sampled tokens of every
+    # source rank are bit-exact against the oracle's own dispatch of them;
+    # every other slot of the buffer holds a real row exactly where the plan
+    # sends one and the sentinel everywhere else
     from load_balancing_planner_b200 import moonep
-    R, S, K, E, B, H, tp = 8, 4096, 8, 256, 32, 7168, 128
-    tk, tpe, _ = problem(R, S, K, E, 2.0, "hot8", seed=0)
-    x = synth.hidden_bf16(R, S, H, seed=0).cuda()
-    w = torch.from_numpy(synth.route_weights(R, S, K, seed=0)).cuda()
-    h = moonep.moonep_create(S, H, K, E, R, B, tp)
+    R, S, K, E, H, tp = 8, 4096, 8, 256, 7168, 128
+    tk, tpe, _ = problem(R, S, K, E, mv, "hot8", seed=0)
+    xh = synth.hidden_bf16(R, S, H, seed=0)
+    wh = synth.route_weights(R, S, K, seed=0)
+    x, w = xh.cuda(), torch.from_numpy(wh).cuda()
+    h = moonep.moonep_create(S, H, K, E, R, B, tp, mode=mode)
     p = gpu_plan(h, tk, tpe)
-    o = oracle.plan(tk, E, B, tp, 0, tpe)
+    o = oracle.plan(tk, E, B, tp, mode, tpe)
     assert np.array_equal(p.dst.cpu().numpy(), o["dst"])
+    if mode:
+        G = E // R
+        home = np.arange(E) // G
+        ovf = [(r, e) for r in range(R) for e in range(E) if home[e] != r and o["row_counts"][r, e] > 0]
+        assert ovf, "the inference case must route some copies through home-row overflow"
     buf = torch.empty((R, h.nvs, H), dtype=torch.int16, device="cuda").fill_(-1).view(torch.bfloat16)
     wn = torch.full((R, h.nvs), float("nan"), dtype=torch.float32, device="cuda")
     moonep.moonep_dispatch(h, p, x, w, buf, wn)
     torch.cuda.synchronize()
-    flat = buf.view(-1, H).view(torch.int16)
+    assert moonep.moonep_read_status(p) == 0
+    flat_buf = buf.view(-1, H).view(torch.int16)
+
+    toks = np.sort(np.random.default_rng(1).choice(S, size=256, replace=False))
+    slots, orow, ow = _sampled_oracle_rows(o, synth.bf16_bits(xh), wh, toks)
+    sl = torch.from_numpy(slots).cuda().long()
+    assert np.array_equal(bits(flat_buf[sl].view(torch.bfloat16)), orow)
+    assert np.array_equal(wn.view(-1)[sl].cpu().numpy().view(np.uint32), ow.view(np.uint32))
+
     d = p.dst.view(-1).long()
     src = x.view(R * S, H).view(torch.int16).repeat_interleave(K, dim=0)
-    assert torch.equal(flat[d], src)
+    assert torch.equal(flat_buf[d], src)
     assert torch.equal(wn.view(-1)[d], w.view(-1))
     untouched = torch.ones(R * h.nvs, dtype=torch.bool, device="cuda")
     untouched[d] = False
-    assert bool((flat[untouched] == -1).all())
+    assert bool((flat_buf[untouched] == -1).all())
     assert bool(torch.isnan(wn.view(-1)[untouched]).all())
     h.close()

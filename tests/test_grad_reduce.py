@@ -73,16 +73,26 @@ def test_reduce_grad_backward_shape_sampled(cuda):
     G0 = [G[:, s:s + 4096].cpu().numpy() for s in starts]
     RB0 = [RB[:, s:s + 4096].cpu().numpy() for s in starts]
     unused = [s for s in range(R * B) if se[s] < 0]
-    sums_before = [RB[s].double().sum().item() for s in unused]
+    assert unused
+    # unused slots: sampled ranges bitwise, and the sum of every slot's 32-bit
+    # patterns (as integers) over the whole slot
+    bitsum_before = RB[unused].view(torch.int32).long().sum(dim=1).cpu()
     moonep.moonep_reduce_grad(h, p, [G.view(E, H, Hp)], [RB.view(R, B, H, Hp)])
     torch.cuda.synchronize()
     assert moonep.moonep_read_status(p) == 0
+    touched = np.unique(se[se >= 0])
+    untouched_e = np.setdiff1d(np.arange(E), touched)
     for s0, g0, rb0 in zip(starts, G0, RB0):
         og, orb = g0.copy(), rb0.copy()
         oracle.reduce_grad(o["slot_expert"], og, orb)
-        assert rel_close(G[:, s0:s0 + 4096].cpu().numpy(), og, RTOL_F32).all()
+        got = G[:, s0:s0 + 4096].cpu().numpy()
+        assert rel_close(got, og, RTOL_F32).all()
+        assert np.array_equal(got[untouched_e].view(np.uint32), g0[untouched_e].view(np.uint32))
+        # the oracle's slots after its reduction: consumed +0.0, unused as before
+        grb = RB[:, s0:s0 + 4096].cpu().numpy()
+        assert np.array_equal(grb.view(np.uint32), orb.view(np.uint32))
     used = [s for s in range(R * B) if se[s] >= 0]
     assert used
     assert bool((RB[used].view(torch.int32) == 0).all())
-    assert [RB[s].double().sum().item() for s in unused] == sums_before
+    assert torch.equal(RB[unused].view(torch.int32).long().sum(dim=1).cpu(), bitsum_before)
     h.close()

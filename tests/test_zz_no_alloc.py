@@ -68,3 +68,46 @@ def test_noalloc_rejects_a_workspace_past_its_array(cuda):
     with pytest.raises(moonep.MoonepError) as e:
         moonep.moonep_plan_noalloc(cfg, tk, None, p)
     assert e.value.code == moonep.ERR_SIZE
+
+
+@pytest.mark.parametrize("mode", [1, 2])
+def test_noalloc_inference_modes_without_router_counts(cuda, mode):
+    # the inference shape (R=8, S=4096, K=8, E=256, B=4) at maxvio 4, where
+    # copies past the B slots overflow to their home rows, with no
+    # tokens_per_expert given: the same plan as the handle path, twice
+    from load_balancing_planner_b200 import moonep
+    dev = torch.device("cuda:0")
+    R, S, K, E, B, tp = 8, 4096, 8, 256, 4, 128
+    tk, _, _ = problem(R, S, K, E, 4.0, "hot8", seed=11)
+    t = torch.from_numpy(tk).to(dev)
+    cfg = moonep.Config(S, 8, K, E, R, B, tp, 0, mode)
+    h = moonep.moonep_create(S, 8, K, E, R, B, tp, mode=mode)
+    ref = _plan_arrays(moonep.moonep_plan(h, t, None))
+    home = np.arange(E) // (E // R)
+    assert any(ref["row_counts"][r, e] > 0 for r in range(R) for e in range(E) if home[e] != r)
+    for _ in range(2):
+        p = moonep.moonep_plan_noalloc(cfg, t, None, moonep.Plan(cfg, dev))
+        torch.cuda.synchronize()
+        _same(_plan_arrays(p), ref)
+    h.close()
+
+
+def test_noalloc_error_then_clean_call(cuda):
+    # a call that fails on the device (an expert id past E) leaves its counts
+    # in the shared array; the next clean call must not see them
+    from load_balancing_planner_b200 import moonep
+    dev = torch.device("cuda:0")
+    R, S, K, E, B, tp = 8, 1024, 8, 64, 8, 128
+    tk, tpe, _ = problem(R, S, K, E, 2.0, "zipf", seed=13)
+    bad = tk.copy()
+    bad[5, 100, 3] = E + 1
+    cfg = moonep.Config(S, 8, K, E, R, B, tp, 0, 0)
+    pb = moonep.moonep_plan_noalloc(cfg, torch.from_numpy(bad).to(dev), torch.from_numpy(tpe).to(dev),
+                                    moonep.Plan(cfg, dev))
+    assert moonep.moonep_read_status(pb) & moonep.STATUS_BAD_EXPERT
+    t, c = torch.from_numpy(tk).to(dev), torch.from_numpy(tpe).to(dev)
+    p = moonep.moonep_plan_noalloc(cfg, t, c, moonep.Plan(cfg, dev))
+    torch.cuda.synchronize()
+    h = moonep.moonep_create(S, 8, K, E, R, B, tp)
+    _same(_plan_arrays(p), _plan_arrays(moonep.moonep_plan(h, t, c)))
+    h.close()
