@@ -800,9 +800,8 @@ def cpu_baseline(w, routes, seed):
     ranks = 4
     b, s = oracle_sample(w, [r["topk_np"] for r in routes], ranks, seed)
     return {"value": round(b / s / 1e9, 3), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"full plan of each of the {len(routes)} routings (all {w['R']} ranks) + dispatch and "
-                      f"combine of every token of {ranks} of {w['R']} source ranks, single-threaded C, "
-                      f"{s:.1f} s", "host_cores_available": os.cpu_count(),
+            "sample": f"plan of {len(routes)} routings + D/C of {ranks} of {w['R']} source ranks, 1 thread, {s:.1f} s",
+            "host_cores_available": os.cpu_count(),
             "legs": oracle_weight_legs(seed)}
 
 
@@ -868,6 +867,47 @@ def run_planner_only(args):
             "back_to_back_us": round(a.elapsed_time(b) * 1e3 / args.steps, 2)}
 
 
+def split_result(result):
+    """(detail, line): the bulky parts of a run (legs, the full per-maxvio
+    sweep, the CPU legs) and the contract line, which keeps every headline
+    figure -- planner us per layer, dispatch+combine GB/s and fraction at each
+    maxvio, the spread -- in a compact form."""
+    line = dict(result)
+    detail = {}
+    if "legs" in line:
+        detail["legs"] = line.pop("legs")
+    sweep = line.pop("sweep", {})
+    detail["sweep"] = sweep
+    line["sweep"] = {mv: {"dc_gbs": v["dc_gbs"], "frac": v["dc_frac_measured"], "plan_us": v["planner_us"],
+                          "plan_ev_us": v["planner_us_event_bracketed"]} for mv, v in sweep.items()}
+    pts = detail.get("legs", {}).get("pages_maxvio_points")
+    if pts:
+        line["pages_points"] = {mv: {"dc_gbs": v["dc_gbs"], "plan_ev_us": v["planner_us_event_bracketed"]}
+                                for mv, v in pts.items()}
+        evs = [v["plan_ev_us"] for v in line["sweep"].values()] + [v["plan_ev_us"] for v in line["pages_points"].values()]
+        line["planner_us_event_bracketed_max"] = max(evs)
+    for k in ("prefetch_weight", "reduce_grad", "group_gemm"):
+        leg = detail.get("legs", {}).get(k)
+        if leg is None:
+            continue
+        if k == "prefetch_weight":
+            line["prefetch_frac"] = {mv: v["frac_measured"] for mv, v in leg["points"].items()}
+        elif k == "reduce_grad":
+            line["reduce_grad_frac"] = leg["frac_measured"]
+        else:
+            line["group_gemm_tflops"] = leg["tflops"]
+    if "cpu_baseline" in line:
+        cb = dict(line["cpu_baseline"])
+        if "legs" in cb:
+            detail["cpu_legs"] = cb.pop("legs")
+        line["cpu_baseline"] = cb
+    if "e2e" in line:
+        e = dict(line["e2e"])
+        detail["e2e_pipelining"] = e.pop("pipelined", None)
+        line["e2e"] = e
+    return detail, line
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -914,7 +954,10 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu:
         result["cpu_baseline"] = cpu_baseline(WORKLOADS[args.config], routes, args.seed)
     if rank == 0:
-        print(json.dumps(result), flush=True)
+        detail, line = split_result(result)
+        # the detail first, on its own line; the contract line stays short and last
+        print(json.dumps({"detail": detail}), flush=True)
+        print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()

@@ -128,3 +128,47 @@ def test_reference_arm_prints_one_contract_line():
         assert k in d, k
     assert d["impl"] == "reference" and d["value"] > 0 and d["steps"] == 1 and d["warmup"] == 3
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_bench_contract_line_is_short_and_keeps_the_headline_figures():
+    # the driver keeps only the tail of stdout: the bulky legs go on an
+    # earlier line, and the last line keeps the planner us, the per-maxvio
+    # fractions and the spread
+    import json
+
+    import bench
+    sweep = {f"{m:g}": dict(realised_maxvio=m, planner_us=18.5, planner_us_event_bracketed=19.9, dispatch_us=740.0,
+                            combine_us=672.0, dc_gbs=5990.1, dc_frac_measured=0.9144, dc_frac_8tbs=0.7488)
+             for m in (0.0, 0.5, 1.0, 2.0, 4.0)}
+    legs = {"pages_maxvio_points": {"10": dict(planner_us_event_bracketed=19.8, dc_gbs=5950.0),
+                                    "20": dict(planner_us_event_bracketed=19.7, dc_gbs=5960.0)},
+            "prefetch_weight": {"points": {"1": dict(frac_measured=0.88), "4": dict(frac_measured=0.92)}},
+            "reduce_grad": dict(frac_measured=0.905), "group_gemm": dict(tflops=1370.2),
+            "rank_local": {"workload": "x" * 3000}}
+    result = {"metric": bench.METRIC, "value": 5900.0, "unit": "GB/s", "n_gpus": 1, "steps": 20, "warmup": 5,
+              "ms_per_step": 1.43, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+              "dtype": "bf16", "data": "synthetic",
+              "config": {"workload": "train: " + bench.describe(bench.WORKLOADS["train"]), "maxvio": [0, 0.5, 1, 2, 4],
+                         "parallelism": "EP=8 emulated on each GPU; independent EP groups per GPU",
+                         "l2": "inputs larger than L2 (hidden rows 470 MB, dispatch buffer 4.7 GB per layer)",
+                         "step": "plan + dispatch + combine of one layer; combine reads the dispatch buffer"},
+              "planner_us": 18.5, "planner_us_event_bracketed": 19.9, "planner_us_back_to_back": 17.0,
+              "dispatch_gbs": 5700.0, "combine_gbs": 6300.0, "dc_frac_measured_min": 0.91, "dc_frac_8tbs_min": 0.74,
+              "spread_vs_maxvio": 0.004, "sweep": sweep, "legs": legs,
+              "roofline": dict(bound="hbm", kernel="dispatch", achieved=5700.1, peak=6551.0, unit="GB/s", frac=0.87,
+                               peak_kind="measured", frac_of_nominal_8tbs=0.71, traffic=4175256576,
+                               bytes_per_launch=4231004160),
+              "gpu_launches": 60, "clocks": {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": [], "samples": 3},
+              "e2e": {"value": 835.6, "unit": "GB/s", "h2d_bytes_per_step": 471867392,
+                      "d2h_bytes_per_step": 469762048, "ms_per_step": 10.1, "steps": 20, "pipelined": "y" * 200},
+              "cpu_baseline": {"value": 1.766, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": "s" * 80,
+                               "host_cores_available": 16, "legs": {"x": 1}}}
+    detail, line = bench.split_result(result)
+    text = json.dumps(line)
+    assert len(text) < 2600, len(text)
+    assert "legs" not in line and "legs" in detail and "legs" not in line["cpu_baseline"]
+    for k in ("planner_us", "planner_us_event_bracketed", "planner_us_event_bracketed_max", "spread_vs_maxvio",
+              "roofline", "cpu_baseline", "e2e", "clocks", "gpu_launches", "pages_points", "prefetch_frac"):
+        assert k in line, k
+    assert set(line["sweep"]) == set(sweep) and line["sweep"]["4"]["frac"] == 0.9144
+    assert line["planner_us_event_bracketed_max"] == 19.9
