@@ -192,8 +192,136 @@ __global__ void __launch_bounds__(32) dispatch_bulk_kernel(const __grid_constant
     __syncwarp();
 }
 
+// ---- dispatch through a deep ring, one producer and one consumer warp --------
+// Warp 0 (lane 0) streams the block's token rows into a ring of NS row stages
+// with bulk loads; warp 1 waits for each row, its lanes k < K resolve the K
+// destination slots (and copy the route weight), and lane 0 writes the row
+// to them with K bulk stores, one bulk group per token.  A stage goes back
+// to the producer once its stores have read it: after committing token i,
+// the consumer waits until at most D groups still read (token i - D is done)
+// and arrives on that stage's "empty" barrier.  So up to D tokens' stores and
+// NS - D loads are in flight per block at any time, and no load waits behind
+// the stores of the token just before it.  Every wait is bounded; a timeout
+// sets MOONEP_STATUS_TIMEOUT, both warps stop, and the block drains the copies
+// it issued before it exits.
+#ifndef MOONEP_RING_NS
+#define MOONEP_RING_NS 14
+#endif
+#ifndef MOONEP_RING_D
+#define MOONEP_RING_D 6
+#endif
+constexpr int kRingNS = MOONEP_RING_NS;
+constexpr int kRingD = MOONEP_RING_D;
+static_assert(kRingD >= 1 && kRingD < kRingNS, "stores in flight must leave a stage for loads");
+
+template <int KT>
+__global__ void __launch_bounds__(64) dispatch_ring_kernel(const __grid_constant__ CopyArgs a) {
+    extern __shared__ __align__(128) uint8_t sm[];
+    __shared__ volatile int s_abort;
+    __shared__ int s_status;
+    pdl_wait();
+    // one read of the plan's status for the whole block (another block may
+    // set BAD_PLAN meanwhile; both warps must take the same branch)
+    if (threadIdx.x == 0) s_status = *a.status;
+    __syncthreads();
+    if (s_status != 0) return;
+    const Dims &d = a.d;
+    const int K = KT > 0 ? KT : d.K;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint32_t rowbytes = (uint32_t)d.H * 2u;
+    const int64_t ntok = a.ntok;
+    const int64_t nslots = (int64_t)d.R * d.nvs;
+    const uint8_t *src = static_cast<const uint8_t *>(a.src);
+    uint8_t *buf = static_cast<uint8_t *>(a.out);
+    const uint32_t stage0 = smem_addr(sm);
+    const uint32_t full0 = smem_addr(sm + (size_t)kRingNS * rowbytes);
+    const uint32_t empty0 = full0 + 8u * kRingNS;
+    const int64_t first = blockIdx.x, step = gridDim.x;
+    const int64_t mine_n = first < ntok ? (ntok - 1 - first) / step + 1 : 0;  // tokens of this block
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kRingNS; ++s) {
+            mbar_init(full0 + 8u * s);
+            mbar_init(empty0 + 8u * s);
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        s_abort = 0;
+    }
+    __syncthreads();
+
+    int64_t issued = 0;  // producer: loads issued
+    if (warp == 0) {
+        if (lane == 0) {
+            for (int64_t i = 0; i < mine_n; ++i) {
+                const int s = (int)(i % kRingNS);
+                if (i >= kRingNS && !mbar_wait(empty0 + 8u * s, (uint32_t)(((i / kRingNS) - 1) & 1))) {
+                    s_abort = 1;
+                    break;
+                }
+                if (s_abort) break;
+                bulk_load(stage0 + s * rowbytes, src + (first + i * step) * rowbytes, rowbytes, full0 + 8u * s);
+                issued = i + 1;
+            }
+        }
+    } else {
+        const uint64_t pol = l2_evict_first_policy();
+        for (int64_t i = 0; i < mine_n; ++i) {
+            const int64_t tok = first + i * step;
+            const int s = (int)(i % kRingNS);
+            uint8_t *mine = nullptr;  // lane k: the row of the token's k-th slot
+            if (lane < K) {
+                const int dk = a.dst[tok * K + lane];
+                if (dk < 0 || dk >= nslots) {
+                    atomicOr(a.status_rw, MOONEP_STATUS_BAD_PLAN);
+                } else {
+                    mine = slot_row(a, buf, dk, rowbytes);
+                    float *wo = slot_weight(a, a.w_out, dk);
+                    if (a.w != nullptr && wo != nullptr) *wo = __ldcs(a.w + tok * K + lane);
+                }
+            }
+            bool ok = true;
+            if (lane == 0) ok = !s_abort && mbar_wait(full0 + 8u * s, (uint32_t)((i / kRingNS) & 1));
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok) {
+                if (lane == 0) s_abort = 1;
+                break;
+            }
+            for (int k = 0; k < K; ++k) {
+                uint8_t *o = shfl_ptr(mine, k);
+                if (lane == 0 && o != nullptr) bulk_store(o, stage0 + s * rowbytes, rowbytes, pol);
+            }
+            if (lane == 0) {
+                bulk_commit();
+                if (i >= kRingD) {
+                    bulk_wait_read<kRingD>();  // token i - D's stores have read its stage
+                    mbar_arrive(empty0 + 8u * (uint32_t)((i - kRingD) % kRingNS));
+                }
+            }
+            __syncwarp();
+        }
+        if (lane == 0) bulk_wait_all();  // the stores must finish before the block's shared memory goes
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && s_abort) {
+        atomicOr(a.status_rw, MOONEP_STATUS_TIMEOUT);
+        // every load still in flight lands before exit: the last one issued
+        // into each stage (the earlier ones completed before it was issued)
+        for (int64_t j = issued - 1; j >= 0 && j >= issued - kRingNS; --j)
+            mbar_wait(full0 + 8u * (uint32_t)(j % kRingNS), (uint32_t)((j / kRingNS) & 1));
+    }
+}
+
+size_t dispatch_ring_smem(const Dims &d) { return (size_t)kRingNS * d.H * 2 + 16 * kRingNS; }
+
 size_t dispatch_bulk_smem(const Dims &d) { return (size_t)kBulkStages * d.H * 2 + 8 * kBulkStages; }
 bool dispatch_use_bulk(const Dims &d) { return (size_t)d.H * 2 >= kBulkMinRow && dispatch_bulk_smem(d) <= 200 * 1024; }
+#ifndef MOONEP_DISPATCH_RING
+#define MOONEP_DISPATCH_RING 1
+#endif
+// the deep ring where its NS row stages fit one block's shared memory
+static bool dispatch_use_ring(const Dims &d) {
+    return MOONEP_DISPATCH_RING && (size_t)d.H * 2 >= kBulkMinRow && dispatch_ring_smem(d) <= 220 * 1024;
+}
 
 // ---- combine -----------------------------------------------------------------
 __device__ __forceinline__ void fma_bf16x8(float (&acc)[8], const uint4 &y, float w) {
@@ -353,6 +481,15 @@ cudaError_t launch_dispatch(const CopyArgs &a, int grid, cudaStream_t st) {
 }
 
 cudaError_t launch_dispatch_bulk(const CopyArgs &a, int grid, cudaStream_t st) {
+    if (dispatch_use_ring(a.d)) {
+        const size_t smem = dispatch_ring_smem(a.d);
+        switch (a.d.K) {
+#define X(k) case k: return launch_pdl_smem(dispatch_ring_kernel<k>, grid, 64, smem, st, a);
+            MOONEP_DISPATCH_CASES(X)
+#undef X
+            default: return launch_pdl_smem(dispatch_ring_kernel<0>, grid, 64, smem, st, a);
+        }
+    }
     const size_t smem = dispatch_bulk_smem(a.d);
     switch (a.d.K) {
 #define X(k) case k: return launch_pdl_smem(dispatch_bulk_kernel<k>, grid, 32, smem, st, a);
@@ -368,11 +505,25 @@ cudaError_t dispatch_bulk_set_smem_limit(size_t bytes) {
     MOONEP_DISPATCH_CASES(X)
     X(0)
 #undef X
+#define X(k) if (e == cudaSuccess) e = cudaFuncSetAttribute(dispatch_ring_kernel<k>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    MOONEP_DISPATCH_CASES(X)
+    X(0)
+#undef X
     return e;
 }
 
 int dispatch_bulk_blocks_per_sm(const Dims &d) {
     int n = 0;
+    if (dispatch_use_ring(d)) {
+        const size_t smem = dispatch_ring_smem(d);
+        switch (d.K) {
+#define X(k) case k: cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, dispatch_ring_kernel<k>, 64, smem); break;
+            MOONEP_DISPATCH_CASES(X)
+#undef X
+            default: cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, dispatch_ring_kernel<0>, 64, smem); break;
+        }
+        return n > 0 ? n : 1;
+    }
     const size_t smem = dispatch_bulk_smem(d);
     switch (d.K) {
 #define X(k) case k: cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, dispatch_bulk_kernel<k>, 32, smem); break;
