@@ -360,6 +360,48 @@ MOONEP_API int moonep_reduce_grad_rank(moonep_handle_t h, const moonep_plan_t *p
                                        moonep_stream_t stream);
 
 /*
+ * ---- Sharing rank buffers between processes ----
+ *
+ * With one process per rank, every rank's dispatch buffer, weight rows and
+ * grad slots must be mapped into its peers (the README's ranks reach them
+ * through one symmetric device mapping: "Weight buffer", "Grad buffer";
+ * MarkTechPost, "Memory contract").  A rank exports the device allocation
+ * behind each of its buffers; the other ranks import it and put the pointer
+ * in the tables of the per-rank calls above.  Works between processes on one
+ * GPU and between GPUs of a node (CUDA IPC; the importer's current device is
+ * the one that accesses the memory).
+ *
+ * The per-rank calls keep bulk (TMA) copies to this GPU's own memory: when a
+ * table holds another GPU's memory, moonep_dispatch_rank,
+ * moonep_prefetch_weight_rank and moonep_reduce_grad_rank use their
+ * plain-load/store kernels for that call (the answer per table is cached on
+ * the handle).  No call waits on another rank: the caller orders the ranks'
+ * phases (e.g. a barrier after every rank's dispatch, before any combine).
+ */
+typedef struct {
+    unsigned char handle[64]; /* the exporting allocation's IPC handle */
+    int64_t offset;           /* the exported pointer's offset in that allocation */
+    int64_t bytes;            /* the allocation's size */
+} moonep_ipc_handle_t;
+
+/* Export the allocation holding the device pointer `ptr` (memory from
+ * cudaMalloc, e.g. a caching allocator's block; not VMM memory).  The handle
+ * is plain bytes: send it to the other processes by any channel. */
+MOONEP_API int moonep_ipc_export(const void *ptr, moonep_ipc_handle_t *out);
+
+/* Map another process's export into this process, on the current device:
+ * *out = the exported pointer here.  Exports from one allocation share one
+ * mapping (reference-counted).  Not for this process's own exports (CUDA
+ * cannot reopen them; use the pointer itself).  ERR_SIZE for an offset
+ * outside the allocation; ERR_CUDA when CUDA refuses the mapping. */
+MOONEP_API int moonep_ipc_import(const moonep_ipc_handle_t *h, void **out);
+
+/* Release one import (the pointer moonep_ipc_import returned); the mapping
+ * closes with its last import.  No kernel may still use it.  ERR_SIZE when
+ * ptr is not an import of this process. */
+MOONEP_API int moonep_ipc_close(void *ptr);
+
+/*
  * moonep_plan without a handle and without allocating: the same plan as
  * moonep_plan for the same cfg and inputs.  (This entry point has no
  * counterpart on the pages; it exists for callers that cannot call cudaMalloc

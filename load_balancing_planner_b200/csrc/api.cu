@@ -5,6 +5,7 @@
 #include <string.h>
 
 #include <mutex>
+#include <new>
 
 #include "moonep_internal.cuh"
 
@@ -30,7 +31,36 @@ struct moonep_handle {
     Workspace ws_rank;  // one-rank planning (moonep_plan_rank): its own barrier counter and parity slots
     uint32_t barrier_polls;     // the planner's grid-barrier poll limit
     uint32_t barrier_withheld;  // arrivals that never come (fault injection for tests; normally 0)
+    int grid_dispatch_vec;      // the vector dispatch kernel's grid (rank tables on other GPUs)
+    // the last pointer tables checked for memory on other GPUs, and the answers
+    static constexpr int kRemoteCache = 4;
+    std::mutex remote_mu;
+    int remote_next;
+    int remote_n[kRemoteCache];
+    const void *remote_tab[kRemoteCache][MOONEP_MAX_PROJ * MOONEP_MAX_R];
+    int remote_ans[kRemoteCache];
 };
+
+// Does any pointer of a rank call's table live on another GPU?  Such tables
+// (peer mappings of a real group on several GPUs) are served with plain
+// loads and stores; bulk copies are kept to this GPU's own memory.  The
+// answers for the last few tables are kept, so a caller that passes the same
+// tables every layer pays for the pointer queries once.
+static bool table_is_remote(moonep_handle_t h, const void *const *tab, int n) {
+    std::lock_guard<std::mutex> lock(h->remote_mu);
+    for (int c = 0; c < moonep_handle::kRemoteCache; ++c)
+        if (n == h->remote_n[c] && memcmp(tab, h->remote_tab[c], sizeof(void *) * (size_t)n) == 0)
+            return h->remote_ans[c] != 0;
+    int remote = 0;
+    for (int i = 0; i < n; ++i)
+        if (on_other_device(tab[i], h->device) == 1) remote = 1;
+    const int c = h->remote_next;
+    h->remote_next = (c + 1) % moonep_handle::kRemoteCache;
+    h->remote_n[c] = n;
+    memcpy(h->remote_tab[c], tab, sizeof(void *) * (size_t)n);
+    h->remote_ans[c] = remote;
+    return remote != 0;
+}
 
 // Handle workspace: [group planning][group GEMM pair table][one-rank planning]
 static size_t pair_table_offset(const Dims &d) { return (workspace_bytes(d) + 255) / 256 * 256; }
@@ -160,29 +190,30 @@ extern "C" int moonep_create(const moonep_config_t *cfg, moonep_handle_t *out) {
     const int rc = check_config(*cfg);
     if (rc != MOONEP_OK) return rc;
 
-    moonep_handle *h = static_cast<moonep_handle *>(calloc(1, sizeof(moonep_handle)));
+    moonep_handle *h = new (std::nothrow) moonep_handle();
     if (!h) return MOONEP_ERR_CUDA;
     h->cfg = *cfg;
     Dims &d = h->d;
     cudaError_t e = cudaGetDevice(&h->device);
     int sms = 0;
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, h->device);
-    if (e != cudaSuccess) { free(h); return fail_cuda(e); }
+    if (e != cudaSuccess) { delete h; return fail_cuda(e); }
     h->sms = (cfg->num_sms > 0 && cfg->num_sms < sms) ? cfg->num_sms : sms;
     int rc2 = prepare_device(h->device);
     if (rc2 == MOONEP_OK) rc2 = plan_dims(*cfg, h->device, &d, &h->grid_plan);
-    if (rc2 != MOONEP_OK) { free(h); return rc2; }
+    if (rc2 != MOONEP_OK) { delete h; return rc2; }
 
     h->bulk_dispatch = dispatch_use_bulk(d);
     h->grid_dispatch = h->sms * (h->bulk_dispatch ? dispatch_bulk_blocks_per_sm(d) : dispatch_blocks_per_sm(d.K));
+    h->grid_dispatch_vec = h->sms * dispatch_blocks_per_sm(d.K);
     h->grid_combine = h->sms * combine_blocks_per_sm(d.K);
     h->grid_weights = h->sms * weights_blocks_per_sm();
 
     const size_t wsb = rank_ws_offset(d) + workspace_bytes(d);
-    if ((e = cudaMalloc(&h->ws_mem, wsb)) != cudaSuccess) { free(h); return fail_cuda(e); }
+    if ((e = cudaMalloc(&h->ws_mem, wsb)) != cudaSuccess) { delete h; return fail_cuda(e); }
     if ((e = cudaMemset(h->ws_mem, 0, wsb)) != cudaSuccess) {
         cudaFree(h->ws_mem);
-        free(h);
+        delete h;
         return fail_cuda(e);
     }
     carve_workspace(d, h->ws_mem, &h->ws);
@@ -197,7 +228,7 @@ extern "C" int moonep_destroy(moonep_handle_t h) {
     if (!h) return MOONEP_OK;
     cudaError_t e = cudaSuccess;
     if (h->ws_mem) e = cudaFree(h->ws_mem);
-    free(h);
+    delete h;
     return e == cudaSuccess ? MOONEP_OK : MOONEP_ERR_CUDA;
 }
 
@@ -308,8 +339,11 @@ extern "C" int moonep_dispatch_rank(moonep_handle_t h, const moonep_plan_t *plan
     a.src = hidden;
     a.w = route_weights;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const cudaError_t e = h->bulk_dispatch ? launch_dispatch_bulk(a, h->grid_dispatch, st)
-                                           : launch_dispatch(a, h->grid_dispatch, st);
+    // bulk stores only into this GPU's memory; rows for other GPUs go as
+    // plain 16-byte stores
+    const bool remote = table_is_remote(h, reinterpret_cast<const void *const *>(a.peer), h->d.R);
+    const cudaError_t e = (h->bulk_dispatch && !remote) ? launch_dispatch_bulk(a, h->grid_dispatch, st)
+                                                        : launch_dispatch(a, h->grid_dispatch_vec, st);
     return e == cudaSuccess ? MOONEP_OK : fail_cuda(e);
 }
 
@@ -413,6 +447,7 @@ static int weight_args_rank(moonep_handle_t h, const moonep_plan_t *plan, int32_
             a->peer[p][q] = x;
         }
     }
+    a->remote = table_is_remote(h, peers, n_proj * h->d.R) ? 1 : 0;
     return MOONEP_OK;
 }
 

@@ -76,6 +76,10 @@ struct CopyArgs {
     float *peer_w[MOONEP_MAX_R];
 };
 
+// 1 when p lives on a device other than `device` (a peer GPU's memory), 0
+// when on `device` (or host-visible), -1 when CUDA cannot tell (ipc.cu)
+int on_other_device(const void *p, int device);
+
 cudaError_t launch_dispatch(const CopyArgs &a, int grid, cudaStream_t st);
 cudaError_t launch_dispatch_bulk(const CopyArgs &a, int grid, cudaStream_t st);
 cudaError_t dispatch_bulk_set_smem_limit(size_t bytes);
@@ -100,6 +104,7 @@ struct WeightArgs {
     // [G,..] (prefetch) or slots [B,..] (reduce_grad).
     int rank;
     const void *peer[MOONEP_MAX_PROJ][MOONEP_MAX_R];
+    int remote;  // some peer tensor lives on another GPU: plain loads and stores only, no bulk copies
 };
 
 cudaError_t launch_prefetch(const WeightArgs &a, int grid, int sms, cudaStream_t st);

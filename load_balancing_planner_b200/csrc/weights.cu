@@ -486,7 +486,7 @@ bool prefetch_use_bulk(const WeightArgs &a) {
 }
 
 cudaError_t launch_prefetch(const WeightArgs &a, int grid, int sms, cudaStream_t st) {
-    if (!prefetch_use_bulk(a)) return launch_w(prefetch_kernel, a, grid, st);
+    if (a.remote || !prefetch_use_bulk(a)) return launch_w(prefetch_kernel, a, grid, st);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(2 * sms));  // two rings per SM
     cfg.blockDim = dim3(kWThreads);
@@ -513,7 +513,7 @@ bool reduce_grad_use_bulk(const WeightArgs &a) {
 }
 
 cudaError_t launch_reduce_grad(const WeightArgs &a, int grid, int sms, cudaStream_t st) {
-    if (!reduce_grad_use_bulk(a)) return launch_w(reduce_grad_kernel, a, grid, st);
+    if (a.remote || !reduce_grad_use_bulk(a)) return launch_w(reduce_grad_kernel, a, grid, st);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(2 * sms));  // two rings per SM
     cfg.blockDim = dim3(kRgThreads);

@@ -12,12 +12,14 @@ each slot's expert from its home rank, and the grad reduction of a home rank
 reads and zeroes the slots of every rank (`moonep_prefetch_weight_rank`,
 `moonep_reduce_grad_rank`).
 
-`RankBuffer` takes those buffers as a list of R tensors.  On a real group
-they are this rank's views of the peers' memory (peer-mapped allocations,
-e.g. from torch's symmetric memory); on one GPU they are R separate local
-allocations, which is how the tests run it.  Argument marshalling only: every
-step runs in the library's kernels, and the gather is a torch.distributed
-collective of the caller's process group.
+`RankBuffer` takes those buffers as a list of R entries: tensors, or device
+pointers of the peers' memory.  With one process per rank, `IpcPeers` maps
+the other ranks' buffers into this process (CUDA IPC, through the library's
+moonep_ipc_export / moonep_ipc_import) and gives the tables; the ranks may
+share one GPU or sit on several GPUs of a node.  Within one process, R
+separate local allocations stand in for the ranks.  Argument marshalling
+only: every step runs in the library's kernels, and the gathers are
+torch.distributed collectives of the caller's process group.
 """
 from __future__ import annotations
 
@@ -38,14 +40,57 @@ def gather_counts(tokens_per_expert: torch.Tensor, group=None) -> torch.Tensor:
     return torch.stack(rows)
 
 
+class IpcPeers:
+    """This rank's tensors, shared with the other ranks of `group` (one
+    process per rank).  Every rank exports the allocation behind each of its
+    tensors, the exports are all-gathered over the group (pickled bytes: a
+    gloo group, or any group that can gather objects), and every rank maps
+    the others' into this process.  `table(i)` lists tensor i of every rank,
+    in group rank order: this rank's own tensor at its own index, the peers'
+    as device pointers.  Tensor i must have the same shape and dtype on every
+    rank.  `close()` releases the mappings once no kernel uses them."""
+
+    def __init__(self, tensors, group=None):
+        self.rank = dist.get_rank(group)
+        self.world = dist.get_world_size(group)
+        self.tensors = list(tensors)
+        mine = [moonep.moonep_ipc_export(t) for t in self.tensors]
+        every = [None] * self.world
+        dist.all_gather_object(every, mine, group=group)
+        self._imports = []
+        self.rows = []
+        for q in range(self.world):
+            if q == self.rank:
+                self.rows.append(list(self.tensors))
+                continue
+            if len(every[q]) != len(self.tensors):
+                raise ValueError(f"rank {q} shared {len(every[q])} tensors, this rank {len(self.tensors)}")
+            row = []
+            for blob in every[q]:
+                ptr = moonep.moonep_ipc_import(blob)
+                self._imports.append(ptr)
+                row.append(ptr)
+            self.rows.append(row)
+
+    def table(self, i: int):
+        """Tensor i of every rank, in rank order (tensors or device pointers)."""
+        return [self.rows[q][i] for q in range(self.world)]
+
+    def close(self) -> None:
+        for ptr in self._imports:
+            moonep.moonep_ipc_close(ptr)
+        self._imports = []
+
+
 class RankBuffer:
     """Rank `rank` of an EP group of `num_ep_ranks`: S tokens, hidden size H,
     top-K over E experts, B prefetch slots.
 
     `hidden_nvs`: the R ranks' dispatched buffers, a list of R [NvS, H] bf16
-    tensors (entry `rank` is this rank's own); `route_weights_nvs` the same
-    for the [NvS] fp32 weights, or None.  NvS is `self.nvs`, known before any
-    buffer exists (`RankBuffer.nvs_of`)."""
+    tensors or device pointers (entry `rank` is this rank's own; e.g.
+    `IpcPeers.table`); `route_weights_nvs` the same for the [NvS] fp32
+    weights, or None.  NvS is `self.nvs`, known before any buffer exists
+    (`RankBuffer.nvs_of`)."""
 
     def __init__(self, S: int, H: int, K: int, E: int, num_ep_ranks: int, rank: int, hidden_nvs,
                  route_weights_nvs=None, token_padding: int = 128, B: int | None = None,

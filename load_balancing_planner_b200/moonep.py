@@ -39,6 +39,10 @@ class PlanSizes(ctypes.Structure):
                 ("dst", "cu_seqlens", "row_counts", "slot_expert", "counts", "assign", "maxvio", "status", "nvs")]
 
 
+class IpcHandle(ctypes.Structure):
+    _fields_ = [("handle", ctypes.c_ubyte * 64), ("offset", ctypes.c_int64), ("bytes", ctypes.c_int64)]
+
+
 class PlanStruct(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("dst", "cu_seqlens", "row_counts", "slot_expert", "counts", "assign", "maxvio", "status")]
@@ -64,6 +68,9 @@ def _load():
         "moonep_plan_status": ([ctypes.POINTER(PlanStruct), ctypes.POINTER(i32)], ctypes.c_int),
         "moonep_plan_sizes": ([ctypes.POINTER(Config), i32, ctypes.POINTER(PlanSizes)], ctypes.c_int),
         "moonep_set_plan_barrier": ([P, ctypes.c_uint32, i32], ctypes.c_int),
+        "moonep_ipc_export": ([P, ctypes.POINTER(IpcHandle)], ctypes.c_int),
+        "moonep_ipc_import": ([ctypes.POINTER(IpcHandle), ctypes.POINTER(P)], ctypes.c_int),
+        "moonep_ipc_close": ([P], ctypes.c_int),
         "moonep_error_string": ([ctypes.c_int], ctypes.c_char_p),
         "moonep_last_error": ([], ctypes.c_char_p),
         "moonep_plan_noalloc": ([ctypes.POINTER(Config), P, P, ctypes.POINTER(PlanStruct), P], ctypes.c_int),
@@ -87,7 +94,7 @@ EXPORTS = ("moonep_create", "moonep_destroy", "moonep_nvs", "moonep_get_config",
            "moonep_read_status", "moonep_error_string", "moonep_last_error", "moonep_plan_noalloc",
            "moonep_group_gemm", "moonep_plan_rank", "moonep_dispatch_rank", "moonep_combine_rank",
            "moonep_prefetch_weight_rank", "moonep_reduce_grad_rank", "moonep_plan_sizes", "moonep_plan_status",
-           "moonep_set_plan_barrier")
+           "moonep_set_plan_barrier", "moonep_ipc_export", "moonep_ipc_import", "moonep_ipc_close")
 NOALLOC_SCRATCH_BYTES = 1 << 20
 
 
@@ -191,6 +198,28 @@ def moonep_set_plan_barrier(h: "Handle", max_polls: int = 0, missing: int = 0):
     _check(lib.moonep_set_plan_barrier(h.ptr, max_polls, missing), "moonep_set_plan_barrier")
 
 
+def moonep_ipc_export(t) -> bytes:
+    """The CUDA IPC export of the allocation holding CUDA tensor t (plain
+    bytes, to send to another process)."""
+    h = IpcHandle()
+    _check(lib.moonep_ipc_export(_ptr(t), ctypes.byref(h)), "moonep_ipc_export")
+    return ctypes.string_at(ctypes.addressof(h), ctypes.sizeof(h))
+
+
+def moonep_ipc_import(blob: bytes) -> int:
+    """Device pointer, in this process, of another process's export."""
+    if len(blob) != ctypes.sizeof(IpcHandle):
+        raise ValueError("not a moonep IPC handle")
+    h = IpcHandle.from_buffer_copy(blob)
+    out = ctypes.c_void_p()
+    _check(lib.moonep_ipc_import(ctypes.byref(h), ctypes.byref(out)), "moonep_ipc_import")
+    return int(out.value)
+
+
+def moonep_ipc_close(ptr: int):
+    _check(lib.moonep_ipc_close(ctypes.c_void_p(ptr)), "moonep_ipc_close")
+
+
 def moonep_create(S, H, K, E, R, B=None, token_padding=128, num_sms=0, mode=TRAINING) -> Handle:
     B = E // R if B is None else B
     cfg = Config(S, H, K, E, R, B, token_padding, num_sms, mode)
@@ -270,7 +299,7 @@ def moonep_combine_rank(h: Handle, plan: Plan, hidden_nvs, route_weights_nvs=Non
     R ranks' buffers (lists as in moonep_dispatch_rank)."""
     _rank_plan(plan, "moonep_combine_rank")
     bufs, wbufs = _rank_tables(h, hidden_nvs, route_weights_nvs)
-    dev = hidden_nvs[0].device
+    dev = torch.device("cuda", torch.cuda.current_device())
     if out is None:
         out = torch.empty((h.S, h.H), dtype=torch.bfloat16, device=dev)
     if gather and route_weights_nvs is not None and gathered_weights is None:
@@ -286,12 +315,14 @@ class PeerTable:
     """The R ranks' same-shaped tensors as one table of device pointers,
     checked once.  Pass it wherever a per-rank call takes a list of R
     tensors: the call then skips the per-tensor checks and the marshalling.
-    The table keeps the tensors alive; their storage must not move."""
+    The table keeps the tensors alive; their storage must not move.  An entry
+    may also be a plain device pointer (int), e.g. a peer process's buffer
+    mapped with moonep_ipc_import, assumed to hold `shape` of `dtype`."""
 
     def __init__(self, tensors, shape, dtype, name="table"):
         self.tensors = list(tensors)
         for t in self.tensors:
-            _expect(t, shape, dtype, name)
+            _expect_entry(t, shape, dtype, name)
         self.arr = _ptr_array(self.tensors)
         self.shape, self.dtype, self.name = tuple(shape), dtype, name
 
@@ -300,6 +331,15 @@ class PeerTable:
 
     def __getitem__(self, i):
         return self.tensors[i]
+
+
+def _expect_entry(t, shape, dtype, name):
+    """A table entry: a tensor of `shape` and `dtype`, or a device pointer (int)."""
+    if isinstance(t, int):
+        if t == 0 or t % 16:
+            raise ValueError(f"{name}: a device pointer must be non-zero and 16-byte aligned")
+        return
+    _expect(t, shape, dtype, name)
 
 
 def _table(h: Handle, x, shape, dtype, name):
@@ -312,7 +352,7 @@ def _table(h: Handle, x, shape, dtype, name):
     if len(x) != h.R:
         raise ValueError("one buffer per rank")
     for b in x:
-        _expect(b, shape, dtype, name)
+        _expect_entry(b, shape, dtype, name)
     return _ptr_array(x)
 
 
@@ -354,11 +394,11 @@ def moonep_combine(h: Handle, plan: Plan, hidden_nvs, route_weights_nvs=None, ou
 
 
 def _ptr_array(ts):
-    arr = (ctypes.c_void_p * len(ts))(*[t.data_ptr() for t in ts])
+    """A C array of device pointers: tensors' data pointers, or ints as given."""
     for t in ts:
-        if not t.is_cuda or not t.is_contiguous():
+        if not isinstance(t, int) and (not t.is_cuda or not t.is_contiguous()):
             raise ValueError("moonep takes contiguous CUDA tensors")
-    return arr
+    return (ctypes.c_void_p * len(ts))(*[t if isinstance(t, int) else t.data_ptr() for t in ts])
 
 
 def moonep_prefetch_weight(h: Handle, plan: Plan, weights, pool, stream=None):
@@ -393,7 +433,7 @@ def _rank_weight_tables(h: Handle, own, peers, own_shape, peer_shape, dtype, nam
         _expect(t, (*own_shape, h.H, Hp), dtype, names[0])
     for row in peers:
         for t in row:
-            _expect(t, (*peer_shape, h.H, Hp), dtype, names[1])
+            _expect_entry(t, (*peer_shape, h.H, Hp), dtype, names[1])
     return _ptr_array(own), _ptr_array([t for row in peers for t in row]), Hp
 
 
