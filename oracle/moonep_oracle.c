@@ -52,6 +52,13 @@
  *     mode 2 (inference, slots by token count): the B received experts with
  *     the most picks on s take the slots (ties: the lower id), in ascending
  *     id; the rest overflow.  [reading; the README leaves the choice open]
+ *     mode 3 (training, fewest copies): step 2 orders the experts of a home
+ *     group by their pick count T_e ascending (ties: the lower id) instead
+ *     of by id, so a donor keeps its smallest experts and the ranges it gives
+ *     away start at its largest ones: a recipient's deficit is covered by as
+ *     few distinct experts (copies) as the donation allows, the fewest
+ *     possible when one donor serves one recipient.  [reading; the README
+ *     calls the planner "near-optimal" without defining the objective]
  *  6. Within a row, picks keep group-sequence order.  Rows are padded to a
  *     multiple of tp (empty rows stay empty); cu_seqlens is the inclusive
  *     running sum of the padded lengths over the E+B rows.  [reading]
@@ -120,13 +127,14 @@ uint16_t oracle_double_to_bf16(double x)
 struct layout {
     int64_t *T, *L, *keep, *estart, *don_amt, *don_start;
     int *don_from, *don_to;
+    int *order; /* [E]: order[h*G + j] = the j-th expert of group h's sequence */
     int ndon;
 };
 
 static void layout_free(struct layout *y)
 {
     free(y->T); free(y->L); free(y->keep); free(y->estart); free(y->don_amt);
-    free(y->don_start); free(y->don_from); free(y->don_to);
+    free(y->don_start); free(y->don_from); free(y->don_to); free(y->order);
 }
 
 /*
@@ -205,10 +213,33 @@ static void plan_layout(int R, int S, int K, int E, int B, int tp, int mode, con
         assign[s * 4 + 3] = (int32_t)don_amt[j];
     }
 
+    /* step 2's order of each group's experts: by id, or in mode 3 by pick
+     * count ascending with ties by id (a plain insertion sort) */
+    int *order = malloc(sizeof(int) * (size_t)E);
+    for (int h = 0; h < R; h++) {
+        int *o = order + (int64_t)h * G;
+        for (int j = 0; j < G; j++) o[j] = h * G + j;
+        if (mode == 3)
+            for (int j = 1; j < G; j++) {
+                int e = o[j], i = j - 1;
+                while (i >= 0 && (T[o[i]] > T[e] || (T[o[i]] == T[e] && o[i] > e))) {
+                    o[i + 1] = o[i];
+                    i--;
+                }
+                o[i + 1] = e;
+            }
+    }
+
     /* start of each expert's run inside its group sequence */
     int64_t *estart = calloc(E, sizeof(int64_t));
-    for (int e = 0; e < E; e++)
-        estart[e] = (e % G == 0) ? 0 : estart[e - 1] + T[e - 1];
+    for (int h = 0; h < R; h++) {
+        int64_t run = 0;
+        for (int j = 0; j < G; j++) {
+            int e = order[(int64_t)h * G + j];
+            estart[e] = run;
+            run += T[e];
+        }
+    }
 
     /* step 5: rows of every rank */
     int *rx_e = malloc(sizeof(int) * (size_t)G);
@@ -270,12 +301,14 @@ static void plan_layout(int R, int S, int K, int E, int B, int tp, int mode, con
     free(rx_n); free(rx_e); free(largeq); free(smallq); free(cur);
     y->T = T; y->L = L; y->keep = keep; y->estart = estart; y->don_amt = don_amt;
     y->don_start = don_start; y->don_from = don_from; y->don_to = don_to; y->ndon = ndon;
+    y->order = order;
 }
 
 /*
  * Inputs: topk [R,S,K] int32 (expert ids), tpe [R,E] int32 or NULL (the
  * router's local counts, checked against the picks).  mode 0 = training
- * (B >= E/R), 1 = inference, 2 = inference with slots by token count.
+ * (B >= E/R), 1 = inference, 2 = inference with slots by token count,
+ * 3 = training with the fewest-copies group order (B >= E/R).
  * Outputs (caller-allocated): dst [R,S,K], cu_seqlens [R,E+B],
  * row_counts [R,E+B], slot_expert [R,B] (-1 = unused), counts [R,E],
  * maxvio [1], assign [R,4] = {kept, donor group or -1, received start in the
@@ -292,7 +325,7 @@ int oracle_plan(int R, int S, int K, int E, int B, int tp, int mode,
     if (R < 1 || S < 1 || K < 1 || E < 1 || E % R || K > E || B < 0 || tp < 1)
         return ORC_BAD_ARGS;
     const int G = E / R;
-    if (mode < 0 || mode > 2 || (mode == 0 && B < G)) return ORC_BAD_ARGS;
+    if (mode < 0 || mode > 3 || ((mode == 0 || mode == 3) && B < G)) return ORC_BAD_ARGS;
     const int64_t C = (int64_t)S * K;
     const int NR = E + B; /* rows per rank */
     const int64_t NvS = oracle_nvs(S, K, E, R, tp);
@@ -332,7 +365,8 @@ int oracle_plan(int R, int S, int K, int E, int B, int tp, int mode,
     int32_t *fill = calloc((size_t)R * NR, sizeof(int32_t));
     for (int h = 0; h < R; h++) {
         int64_t g = 0;
-        for (int e = h * G; e < (h + 1) * G; e++)
+        for (int jj = 0; jj < G; jj++) {
+            const int e = y.order[(int64_t)h * G + jj];
             for (int r = 0; r < R; r++)
                 for (int t = 0; t < S; t++)
                     for (int k = 0; k < K; k++) {
@@ -354,6 +388,7 @@ int oracle_plan(int R, int S, int K, int E, int B, int tp, int mode,
                         fill[ri]++;
                         g++;
                     }
+        }
     }
 
     free(fill);
@@ -385,7 +420,7 @@ int oracle_plan_rank(int R, int S, int K, int E, int B, int tp, int mode, int ra
     if (R < 1 || S < 1 || K < 1 || E < 1 || E % R || K > E || B < 0 || tp < 1 || rank < 0 || rank >= R)
         return ORC_BAD_ARGS;
     const int G = E / R;
-    if (mode < 0 || mode > 2 || (mode == 0 && B < G)) return ORC_BAD_ARGS;
+    if (mode < 0 || mode > 3 || ((mode == 0 || mode == 3) && B < G)) return ORC_BAD_ARGS;
     const int64_t C = (int64_t)S * K;
     const int NR = E + B;
     const int64_t NvS = oracle_nvs(S, K, E, R, tp);

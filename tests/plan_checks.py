@@ -57,7 +57,7 @@ def check_plan(topk, p, E, B, tp, mode, nvs=None):
             else:
                 assert rc[r, E + b] > 0, "a used slot holds picks"
         remote_rows = [e for e in range(E) if e // G != r and rc[r, e] > 0]  # overflow rows
-        if mode == 0:
+        if mode in (0, 3):
             assert not remote_rows, "training never reads a remote home row"
         remote_experts = set(used.tolist()) | set(remote_rows)
         groups = {e // G for e in remote_experts}

@@ -87,6 +87,9 @@ CASES = [
     dict(R=4, S=333, K=3, E=24, B=0, tp=16, mode=1, mv=1.5, profile="hot8"),
     dict(R=1, S=100, K=4, E=16, B=16, tp=8, mode=0, mv=1.0, profile="zipf"),
     dict(R=8, S=64, K=1, E=8, B=1, tp=1, mode=0, mv=3.0, profile="boost0"),
+    dict(R=8, S=1024, K=8, E=64, B=8, tp=128, mode=3, mv=2.0, profile="zipf"),
+    dict(R=4, S=333, K=3, E=24, B=6, tp=16, mode=3, mv=1.5, profile="hot8"),
+    dict(R=8, S=4096, K=8, E=256, B=32, tp=128, mode=3, mv=0.5, profile="hot8"),
 ]
 
 
@@ -121,8 +124,8 @@ def small_problem(draw):
     K = draw(st.integers(1, min(E, 4)))
     S = draw(st.integers(1, 12))
     tp = draw(st.integers(1, 4))
-    mode = draw(st.integers(0, 2))
-    B = draw(st.integers(G, G + 1)) if mode == 0 else draw(st.integers(0, G))
+    mode = draw(st.integers(0, 3))
+    B = draw(st.integers(G, G + 1)) if mode in (0, 3) else draw(st.integers(0, G))
     seed = draw(st.integers(0, 2 ** 31 - 1))
     hot = draw(st.floats(0.0, 4.0))
     g = np.random.default_rng(seed)
@@ -139,8 +142,30 @@ def test_plan_invariants_random(prob):
     p = oracle.plan(tk, E, B, tp, mode)
     assert p["status"] == 0
     check_plan(tk, p, E, B, tp, mode)
-    if mode:
+    if mode in (1, 2):
         _check_slot_choice(p, E, B, tk.shape[0], by_count=mode == 2)
+    if mode == 3:
+        _check_largest_experts_donated(tk, p, E)
+
+
+def _check_largest_experts_donated(tk, p, E):
+    """Mode 3: a donor keeps its smallest experts.  Ordering a group's experts
+    by (count, id), every expert the donor keeps whole comes before every
+    expert it gives away whole, and at most one expert is split."""
+    R = tk.shape[0]
+    G = E // R
+    T = np.bincount(tk.reshape(-1), minlength=E)
+    rc = p["row_counts"]
+    for h in range(R):
+        if not any(p["assign"][s, 1] == h for s in range(R)):
+            continue
+        kept = {e: int(rc[h, e]) for e in range(h * G, (h + 1) * G)}
+        whole_kept = [(T[e], e) for e, n in kept.items() if T[e] and n == T[e]]
+        whole_given = [(T[e], e) for e, n in kept.items() if T[e] and n == 0]
+        split = [e for e, n in kept.items() if 0 < n < T[e]]
+        assert len(split) <= 1
+        if whole_kept and whole_given:
+            assert max(whole_kept) < min(whole_given), (h, whole_kept, whole_given)
 
 
 def _check_slot_choice(p, E, B, R, by_count):
@@ -234,11 +259,12 @@ def _sorted_layout(tk, E, B, tp, h, G):
     return want
 
 
+@pytest.mark.parametrize("mode", [0, 3])
 @pytest.mark.parametrize("R,S,K,E,tp", [(8, 1024, 8, 64, 128), (4, 96, 4, 16, 8), (2, 64, 2, 8, 1)])
-def test_balanced_plan_is_stable_argsort(R, S, K, E, tp):
+def test_balanced_plan_is_stable_argsort(R, S, K, E, tp, mode):
     tk, mv, _ = synth.routing(R, S, K, E, 0.0, seed=5)
     G = E // R
-    p = oracle.plan(tk, E, G, tp)
+    p = oracle.plan(tk, E, G, tp, mode)
     assert p["status"] == 0 and copies_of(p, E, G, R) == 0
     assert np.all(p["assign"][:, 1] == -1)
     flat = p["dst"].reshape(-1)
@@ -519,6 +545,42 @@ def test_bruteforce_min_copies_tiny():
     assert gaps.max() <= 1  # observed on this tiny space; reported, not a page claim
 
 
+def test_fewest_copies_mode_reaches_the_bruteforce_minimum_tiny():
+    # R=2, E=4, S=3, K=1, every routing: with one donor and one recipient,
+    # giving away the largest experts first covers the deficit with the
+    # fewest experts, so mode 3's copy count is the brute-force minimum
+    R, E, S, K = 2, 4, 3, 1
+    for picks in itertools.product(range(E), repeat=R * S * K):
+        tk = np.array(picks, np.int32).reshape(R, S, K)
+        p = oracle.plan(tk, E, E // R, 1, 3)
+        assert p["status"] == 0
+        check_plan(tk, p, E, E // R, 1, 3)
+        assert copies_of(p, E, E // R, R) == _min_copies_bruteforce(tk, E, R), picks
+
+
+def test_fewest_copies_mode_with_equal_counts_is_the_id_order():
+    # within each group all experts have one count: the count order is the id
+    # order (ties by id), so mode 3 plans exactly as mode 0
+    R, S, K, E = 2, 8, 1, 4
+    # T = [3, 3, 5, 5]: group 0 under-loaded (6), group 1 over-loaded (10)
+    picks = [0, 0, 0, 1, 1, 1, 2, 2, 2, 2, 2, 3, 3, 3, 3, 3]
+    tk = np.array(picks, np.int32).reshape(R, S, K)
+    a, b = oracle.plan(tk, E, 2, 2, 0), oracle.plan(tk, E, 2, 2, 3)
+    assert a["status"] == b["status"] == 0
+    assert np.any(a["assign"][:, 1] >= 0), "the case must donate"
+    for k in ("dst", "cu_seqlens", "row_counts", "slot_expert", "assign"):
+        assert np.array_equal(a[k], b[k]), k
+
+
+def test_fewest_copies_mode_never_copies_more_with_one_donor_per_recipient_pair():
+    # where the alias chain makes a single donation (R=2), mode 3 never makes
+    # more copies than mode 0; across larger groups its count is reported
+    for seed in range(40):
+        tk, _, _ = synth.routing(2, 64, 4, 16, 0.5 + 0.5 * (seed % 5), "hot8", seed=seed)
+        a, b = oracle.plan(tk, 16, 8, 4, 0), oracle.plan(tk, 16, 8, 4, 3)
+        assert copies_of(b, 16, 8, 2) <= copies_of(a, 16, 8, 2)
+
+
 # ------------------------------------------------ one rank's share of the plan
 @pytest.mark.parametrize("R,S,K,E,B,tp,mode,mv,profile", [
     (8, 1024, 8, 64, 8, 128, 0, 2.0, "zipf"),
@@ -529,6 +591,8 @@ def test_bruteforce_min_copies_tiny():
     (8, 512, 8, 64, 2, 128, 2, 4.0, "hot8"),
     (2, 100, 32, 64, 32, 4, 0, 0.5, "zipf"),
     (16, 64, 4, 64, 4, 8, 0, 6.0, "hot8"),
+    (8, 1024, 8, 64, 8, 128, 3, 2.0, "zipf"),
+    (3, 1000, 3, 24, 8, 16, 3, 1.5, "hot8"),
 ])
 def test_rank_share_is_the_slice_of_the_group_plan(R, S, K, E, B, tp, mode, mv, profile):
     # The group plan walks every group sequence with all ranks' picks; a

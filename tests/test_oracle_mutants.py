@@ -23,8 +23,17 @@ MUTANTS = {
     "drained donor served last": (
         "if (cur[l] < C) { lh++; smallq[--sh] = l; }", "if (cur[l] < C) { lh++; smallq[st++] = l; }"),
     "expert start off by one term": (
-        "estart[e] = (e % G == 0) ? 0 : estart[e - 1] + T[e - 1];",
-        "estart[e] = (e % G == 0) ? 0 : estart[e - 1] + T[e];"),
+        "            estart[e] = run;\n            run += T[e];",
+        "            run += T[e];\n            estart[e] = run;"),
+    "fewest-copies order descending": (
+        "while (i >= 0 && (T[o[i]] > T[e] || (T[o[i]] == T[e] && o[i] > e))) {",
+        "while (i >= 0 && (T[o[i]] < T[e] || (T[o[i]] == T[e] && o[i] > e))) {"),
+    "fewest-copies ties to the higher id": (
+        "while (i >= 0 && (T[o[i]] > T[e] || (T[o[i]] == T[e] && o[i] > e))) {",
+        "while (i >= 0 && (T[o[i]] > T[e] || (T[o[i]] == T[e] && o[i] < e))) {"),
+    "fewest-copies walk in id order": (
+        "            const int e = y.order[(int64_t)h * G + jj];",
+        "            const int e = h * G + jj;"),
     "cu_seqlens exclusive": (
         "cu_seqlens[(int64_t)s * NR + i] = (int32_t)run;\n",
         "cu_seqlens[(int64_t)s * NR + i] = (int32_t)(run - (n ? pad_up(n, tp) : 0));\n"),
