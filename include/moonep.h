@@ -86,8 +86,13 @@ typedef struct CUstream_st *moonep_stream_t;
  *                      inference where the B slots go to the received experts
  *                      with the most picks on the rank (ties: lower id), so
  *                      the home-row overflow carries the fewest tokens (the
- *                      README leaves this choice open).  Slots are in
- *                      ascending expert id in every mode.
+ *                      README leaves this choice open); 3 = training with
+ *                      the fewest copies: a home group's picks are ordered
+ *                      by expert pick count (ascending, ties by id) instead
+ *                      of by id, so a donor gives away its largest experts
+ *                      and every recipient's range spans as few experts as
+ *                      the donation allows (B >= E/R, as in mode 0).  Slots
+ *                      are in ascending expert id in every mode.
  */
 typedef struct {
     int32_t S, H, K, E, R, B, token_padding, num_sms, mode;
@@ -148,7 +153,8 @@ MOONEP_API int moonep_plan_sizes(const moonep_config_t *cfg, int32_t one_rank, m
  * Validate cfg and create a handle on the current device; allocates the
  * planning workspace (cudaMalloc, a few hundred KB).  Rejects (ERR_CONFIG):
  * E % R != 0, K > E, H % 8 != 0, training with B < E/R, sizes past the
- * MOONEP_MAX_* limits, R*S*K or R*NvS at or above 2^31.  *out is NULL on error.
+ * MOONEP_MAX_* limits, R*S*K or R*NvS at or above 2^31, a mode outside 0..3.
+ * *out is NULL on error.
  */
 MOONEP_API int moonep_create(const moonep_config_t *cfg, moonep_handle_t *out);
 

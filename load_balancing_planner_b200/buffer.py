@@ -54,9 +54,11 @@ class Buffer:
     `num_sms` caps the SMs of the copy kernels; None uses every SM (the
     pages default to 32 because their communication kernels share the GPU
     with expert GEMMs; an emulated layer is a pure HBM copy and wants all).
-    `mode` is moonep.TRAINING, moonep.INFERENCE (overflow home rows; slots
-    to the first B received experts) or moonep.INFERENCE_BY_COUNT (slots to
-    the B received experts with the most picks).
+    `mode` is moonep.TRAINING, moonep.TRAINING_FEWEST_COPIES (a donor gives
+    away its largest experts, so recipients hold fewer copies),
+    moonep.INFERENCE (overflow home rows; slots to the first B received
+    experts) or moonep.INFERENCE_BY_COUNT (slots to the B received experts
+    with the most picks).
     """
 
     def __init__(self, S: int, H: int, K: int, E: int, num_ep_ranks: int, num_sms: int | None = None,

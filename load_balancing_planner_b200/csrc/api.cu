@@ -106,8 +106,8 @@ int check_config(const moonep_config_t &c) {
     if (c.K < 1 || c.K > MOONEP_MAX_K || c.K > c.E) return MOONEP_ERR_CONFIG;
     if (c.S < 1 || c.H < 8 || c.H % 8 != 0) return MOONEP_ERR_CONFIG;
     if (c.B < 0 || c.token_padding < 1 || c.num_sms < 0) return MOONEP_ERR_CONFIG;
-    if (c.mode < 0 || c.mode > 2) return MOONEP_ERR_CONFIG;
-    if (c.mode == 0 && c.B < c.E / c.R) return MOONEP_ERR_CONFIG;
+    if (c.mode < 0 || c.mode > 3) return MOONEP_ERR_CONFIG;
+    if ((c.mode == 0 || c.mode == 3) && c.B < c.E / c.R) return MOONEP_ERR_CONFIG;
     if ((int64_t)c.R * c.B > 4096 || c.E + (int64_t)c.B > (int64_t)1 << 20) return MOONEP_ERR_CONFIG;
     if ((int64_t)c.R * c.S * c.K >= ((int64_t)1 << 31)) return MOONEP_ERR_CONFIG;
     if (c.token_padding > (1 << 20)) return MOONEP_ERR_CONFIG;

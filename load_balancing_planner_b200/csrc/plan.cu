@@ -4,7 +4,8 @@
 // remote home group per rank in training, overflow experts read from their
 // home rows in inference, padded cu_seqlens[E+B] -- but print no rule.  The
 // rule implemented here is this library's reading: the group sequence of home
-// rank h lists its picks by (expert, source rank, token); an alias chain over
+// rank h lists its picks by (expert, source rank, token), experts in id order
+// (or, in the fewest-copies mode, by pick count); an alias chain over
 // the group loads decides who gives how much to whom; a donor keeps the prefix
 // of its sequence and gives consecutive ranges after it; a recipient's copied
 // experts take its slots in ascending id, overflow rows past B (inference).
@@ -632,9 +633,35 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
         }
     }
     PLAN_TRACE(10);
-    // expert starts inside their group sequences (warps 1.., one home group
-    // each, while warp 0 runs the alias chain)
-    if (w >= 1) {
+    // expert starts inside their group sequences (warps 1.., while warp 0
+    // runs the alias chain).  Mode 3 (fewest copies) orders a group by pick
+    // count, ties by id: an expert starts after every expert of its group
+    // that sorts before it, one pass over the group per expert.
+    if (d.mode == 3 && G <= 32) {
+        // one warp per group, expert j on lane j: the group's counts are
+        // passed round the warp once
+        for (int h = w - 1; w >= 1 && h < R; h += kPlanWarps - 1) {
+            const int te = lane < G ? T[h * G + lane] : 0;
+            int sum = 0;
+            // not unrolled: this code runs once per block and is fetched cold
+#pragma unroll 1
+            for (int m = 0; m < 32; ++m) {
+                const int tm = __shfl_sync(0xffffffffu, te, m);
+                sum += (m < G && (tm < te || (tm == te && m < lane))) ? tm : 0;
+            }
+            if (lane < G) es[h * G + lane] = sum;
+        }
+    } else if (d.mode == 3) {
+        for (int e = tid - 32; w >= 1 && e < E; e += kPlanThreads - 32) {
+            const int g0 = e - e % G, te = T[e];
+            int sum = 0;
+            for (int m = g0; m < g0 + G; ++m) {
+                const int tm = T[m];
+                if (tm < te || (tm == te && m < e)) sum += tm;
+            }
+            es[e] = sum;
+        }
+    } else if (w >= 1) {
         for (int h = w - 1; h < R; h += kPlanWarps - 1) {
             int carry = 0;
             for (int j0 = 0; j0 < G; j0 += 32) {

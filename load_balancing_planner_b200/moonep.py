@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(_PKG, "libmoonep.so")
 OK, ERR_NULL, ERR_CONFIG, ERR_ALIGN, ERR_CUDA, ERR_SIZE = 0, -1, -2, -3, -4, -5
 STATUS_BAD_EXPERT, STATUS_DUP_EXPERT, STATUS_COUNT_MISMATCH, STATUS_BAD_PLAN, STATUS_TIMEOUT = 1, 2, 4, 8, 16
 MAX_R, MAX_E, MAX_K, MAX_PROJ = 64, 4096, 32, 8
-TRAINING, INFERENCE, INFERENCE_BY_COUNT = 0, 1, 2
+TRAINING, INFERENCE, INFERENCE_BY_COUNT, TRAINING_FEWEST_COPIES = 0, 1, 2, 3
 
 
 class MoonepError(RuntimeError):

@@ -51,7 +51,8 @@ def test_error_strings():
     dict(E=8192, R=8),           # E past the limit
     dict(K=33, E=64),            # K past the limit
     dict(token_padding=0),
-    dict(mode=3),
+    dict(mode=4),
+    dict(B=1, mode=3),           # the fewest-copies training mode needs B >= E/R too
     dict(S=0),
     dict(S=1 << 20, K=32, R=64, E=256),  # R*S*K >= 2^31
 ])

@@ -33,6 +33,12 @@ CASES = [
     # 16384 tokens per rank: chunks grow until every block is resident, and
     # each block reads many earlier chunk rows of its rank
     ("long_seq", 8, 16384, 8, 256, 32, 128, 0, "hot8", [2.0]),
+    # training with the fewest copies: groups ordered by pick count
+    ("fewest_train", 8, 4096, 8, 256, 32, 128, 3, "hot8", [0.0, 0.5, 1.0, 2.0, 4.0, 10.0, 20.0]),
+    ("fewest_zipf", 8, 1024, 8, 64, 8, 128, 3, "zipf", [0.5, 2.0]),
+    ("fewest_ragged", 3, 1000, 3, 24, 8, 16, 3, "hot8", [1.5]),
+    ("fewest_many_ranks", 64, 40, 4, 256, 4, 8, 3, "hot8", [3.0]),
+    ("fewest_wide_e", 4, 600, 8, 1024, 256, 64, 3, "hot8", [2.0]),
 ]
 
 
@@ -145,3 +151,24 @@ def test_inference_slot_rules_differ_on_gpu_as_in_the_oracle(cuda):
         assert_plans_equal(got[mode], oracle.plan(tk, E, B, tp, mode, tpe))
         h.close()
     assert not np.array_equal(got[1]["slot_expert"], got[2]["slot_expert"])
+
+
+def test_fewest_copies_mode_makes_fewer_copies_at_the_training_shape(cuda):
+    # the two training modes on the same routing (R=8, S=4096, K=8, E=256,
+    # B=32): both bit-exact against the oracle; mode 3 never holds more
+    # copies in total over the sweep, and fewer at some maxvio
+    from load_balancing_planner_b200 import moonep
+    from tests.plan_checks import copies_of
+    R, S, K, E, B, tp = 8, 4096, 8, 256, 32, 128
+    h0 = moonep.moonep_create(S, 8, K, E, R, B, tp, mode=0)
+    h3 = moonep.moonep_create(S, 8, K, E, R, B, tp, mode=3)
+    tot0 = tot3 = 0
+    for mv in (0.5, 1.0, 2.0, 4.0, 10.0, 20.0):
+        tk, tpe, _ = problem(R, S, K, E, mv, "hot8", seed=5)
+        a, b = plan_to_numpy(gpu_plan(h0, tk, tpe)), plan_to_numpy(gpu_plan(h3, tk, tpe))
+        assert_plans_equal(b, oracle.plan(tk, E, B, tp, 3, tpe))
+        tot0 += copies_of(a, E, B, R)
+        tot3 += copies_of(b, E, B, R)
+    assert tot3 < tot0, (tot3, tot0)
+    h0.close()
+    h3.close()

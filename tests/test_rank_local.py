@@ -45,6 +45,8 @@ CASES = [
     ("k32", 2, 100, 32, 64, 32, 4, 0, "zipf", 0.5),
     ("many_ranks", 64, 40, 4, 256, 4, 8, 0, "hot8", 3.0),
     ("long_seq", 8, 16384, 8, 256, 32, 128, 0, "hot8", 2.0),
+    ("fewest_train", 8, 4096, 8, 256, 32, 128, 3, "hot8", 2.0),
+    ("fewest_ragged", 3, 1000, 3, 24, 8, 16, 3, "hot8", 1.5),
 ]
 
 
