@@ -265,6 +265,114 @@ __global__ void __launch_bounds__(kWThreads) prefetch_bulk_kernel(const __grid_c
     bulk_wait_all();
 }
 
+// Deep-ring variant of the bulk prefetch, one block per SM: after the block
+// has built the slot lists, warp 0 (lane 0) streams the block's 32 KB pieces
+// into a ring of kPfRing stages with bulk loads, and warp 1 (lane 0) writes
+// each piece to every slot holding its expert with bulk stores, one bulk
+// group per piece, handing a stage back once its stores have read it (up to
+// kPfInFlight pieces' stores in flight).  No load waits behind the stores of
+// the piece before it.  Waits are bounded; a timeout sets
+// MOONEP_STATUS_TIMEOUT, both warps stop, and the loads in flight land
+// before the block exits.
+#ifndef MOONEP_PF_RING
+#define MOONEP_PF_RING 4
+#endif
+constexpr int kPfRing = MOONEP_PF_RING;
+constexpr int kPfInFlight = kPfRing / 2;
+
+__global__ void __launch_bounds__(kWThreads) prefetch_ring_kernel(const __grid_constant__ WeightArgs a) {
+    __shared__ volatile int s_abort;
+    __shared__ int s_status;
+    pdl_wait();
+    // one read of the plan's status for the whole block (another block may
+    // flag BAD_PLAN meanwhile; every thread must take the same branch)
+    if (threadIdx.x == 0) s_status = *a.status;
+    __syncthreads();
+    if (s_status != 0) return;
+    extern __shared__ __align__(128) int32_t wsm[];
+    const int RB = a.d.R * a.d.B;
+    int32_t *se = wsm, *nxt = wsm + RB, *lead = wsm + 2 * RB;
+    const int nlead = build_slot_lists(a, se, nxt, lead, false);  // block-uniform result
+    if (nlead <= 0) return;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (warp > 1) return;
+    uint8_t *stages = reinterpret_cast<uint8_t *>(wsm) + ((sizeof(int32_t) * 3 * (size_t)RB + 127) & ~(size_t)127);
+    const uint32_t stage0 = smem_addr(stages);
+    const uint32_t full0 = stage0 + kPfRing * kPfTile;
+    const uint32_t empty0 = full0 + 8u * kPfRing;
+    const uint64_t bytes_per = (uint64_t)a.hhp * 2;  // one expert matrix, bf16
+    const int64_t ntiles = (int64_t)((bytes_per + kPfTile - 1) / kPfTile);
+    const int64_t units = (int64_t)a.n_proj * nlead * ntiles;
+    const int64_t first = blockIdx.x, step = gridDim.x;
+    const int64_t mine_n = first < units ? (units - 1 - first) / step + 1 : 0;
+    auto piece = [&](int64_t i, int &p, int &s, uint64_t &off, uint32_t &n) {
+        const int64_t u = first + i * step;
+        p = (int)(u / ((int64_t)nlead * ntiles));
+        const int64_t rem = u - (int64_t)p * nlead * ntiles;
+        s = lead[rem / ntiles];
+        off = (uint64_t)(rem % ntiles) * kPfTile;
+        n = (uint32_t)min((uint64_t)kPfTile, bytes_per - off);
+    };
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < kPfRing; ++st) {
+            mbar_init(full0 + 8u * st);
+            mbar_init(empty0 + 8u * st);
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        s_abort = 0;
+    }
+    // warps 0 and 1 only: named barrier 1 over 64 threads
+    asm volatile("bar.sync 1, 64;" ::: "memory");
+    int64_t issued = 0;
+    if (warp == 0 && lane == 0) {
+        for (int64_t i = 0; i < mine_n; ++i) {
+            const int st = (int)(i % kPfRing);
+            if (i >= kPfRing && !mbar_wait(empty0 + 8u * st, (uint32_t)(((i / kPfRing) - 1) & 1))) {
+                s_abort = 1;
+                break;
+            }
+            if (s_abort) break;
+            int p, s;
+            uint64_t off;
+            uint32_t n;
+            piece(i, p, s, off, n);
+            bulk_load(stage0 + st * kPfTile,
+                      reinterpret_cast<const uint8_t *>(expert_at(a, a.src[p], p, se[s], bytes_per, true)) + off, n,
+                      full0 + 8u * st);
+            issued = i + 1;
+        }
+    } else if (warp == 1 && lane == 0) {
+        const uint64_t pol = l2_evict_first_policy();
+        for (int64_t i = 0; i < mine_n; ++i) {
+            const int st = (int)(i % kPfRing);
+            if (s_abort || !mbar_wait(full0 + 8u * st, (uint32_t)((i / kPfRing) & 1))) {
+                s_abort = 1;
+                break;
+            }
+            int p, s;
+            uint64_t off;
+            uint32_t n;
+            piece(i, p, s, off, n);
+            for (int j = s; j >= 0; j = nxt[j])
+                bulk_store(reinterpret_cast<uint8_t *>(slot_at(a, a.dst[p], p, j, bytes_per, false)) + off,
+                           stage0 + st * kPfTile, n, pol);
+            bulk_commit();
+            if (i >= kPfInFlight) {
+                bulk_wait_read<kPfInFlight>();  // piece i - kPfInFlight's stores have read its stage
+                mbar_arrive(empty0 + 8u * (uint32_t)((i - kPfInFlight) % kPfRing));
+            }
+        }
+        bulk_wait_all();  // the stores finish before the block's shared memory goes
+    }
+    asm volatile("bar.sync 1, 64;" ::: "memory");
+    if (threadIdx.x == 0 && s_abort) {
+        atomicOr(a.status, MOONEP_STATUS_TIMEOUT);
+        // the last load issued into each stage lands before exit
+        for (int64_t j = issued - 1; j >= 0 && j >= issued - kPfRing; --j)
+            mbar_wait(full0 + 8u * (uint32_t)(j % kPfRing), (uint32_t)((j / kPfRing) & 1));
+    }
+}
+
 // a.src[p] = reduce buffer [R*B, H*Hp] (read, then zeroed), a.dst[p] = grads [E, H*Hp].
 __global__ void __launch_bounds__(kWThreads) reduce_grad_kernel(const __grid_constant__ WeightArgs a) {
     pdl_wait();
@@ -485,8 +593,29 @@ bool prefetch_use_bulk(const WeightArgs &a) {
     return aligned && a.hhp * 2 >= kPfTile && prefetch_bulk_smem(a) <= 110 * 1024;
 }
 
+static size_t prefetch_ring_smem(const WeightArgs &a) {
+    return ((weights_smem(a) + 127) & ~(size_t)127) + kPfRing * (size_t)kPfTile + 16 * kPfRing;
+}
+
+#ifndef MOONEP_PF_USE_RING
+#define MOONEP_PF_USE_RING 1
+#endif
+
 cudaError_t launch_prefetch(const WeightArgs &a, int grid, int sms, cudaStream_t st) {
     if (a.remote || !prefetch_use_bulk(a)) return launch_w(prefetch_kernel, a, grid, st);
+    if (MOONEP_PF_USE_RING && prefetch_ring_smem(a) <= 220 * 1024) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)sms);  // one deep ring per SM
+        cfg.blockDim = dim3(kWThreads);
+        cfg.dynamicSmemBytes = prefetch_ring_smem(a);
+        cfg.stream = st;
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        at[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = at;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, prefetch_ring_kernel, a);
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(2 * sms));  // two rings per SM
     cfg.blockDim = dim3(kWThreads);
@@ -539,6 +668,7 @@ size_t weights_static_smem_bytes() {
     if (cudaFuncGetAttributes(&fa, prefetch_kernel) == cudaSuccess) m = fa.sharedSizeBytes;
     if (cudaFuncGetAttributes(&fa, reduce_grad_kernel) == cudaSuccess && fa.sharedSizeBytes > m) m = fa.sharedSizeBytes;
     if (cudaFuncGetAttributes(&fa, prefetch_bulk_kernel) == cudaSuccess && fa.sharedSizeBytes > m) m = fa.sharedSizeBytes;
+    if (cudaFuncGetAttributes(&fa, prefetch_ring_kernel) == cudaSuccess && fa.sharedSizeBytes > m) m = fa.sharedSizeBytes;
     if (cudaFuncGetAttributes(&fa, reduce_grad_bulk_kernel) == cudaSuccess && fa.sharedSizeBytes > m)
         m = fa.sharedSizeBytes;
     return m;
@@ -548,6 +678,8 @@ cudaError_t weights_set_smem_limit(size_t bytes) {
     cudaError_t e = cudaFuncSetAttribute(prefetch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(prefetch_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(prefetch_ring_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(reduce_grad_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e != cudaSuccess) return e;
