@@ -18,9 +18,16 @@ Also measured in the same run (unless switched off):
   * cpu_baseline: the CPU oracle on a bounded sample, one host core.
 
 `--impl reference` times the CPU oracle itself on the same workload (see the
-reference-arm section below).  Multi-GPU (`torchrun ... --gpus N`): every rank
-runs its own independent EP group (weak scaling, no data-path collective);
-time is the max over ranks.
+reference-arm section below).
+
+Multi-GPU (`torchrun ... --gpus N`, N > 1): the workload's EP group of R=8
+ranks is sharded over the N processes, R/N ranks per process and GPU (one EP
+rank per process at N = 8).  Each process owns its ranks' dispatch buffers
+and maps its peers' with CUDA IPC; per step it all-gathers the router counts,
+plans its ranks' shares, dispatches their rows into the owners' buffers over
+NVLink, and after a barrier combines its tokens from them (strong scaling:
+the layer is fixed, N GPUs share it).  Time is the max over processes.
+`--replicas` runs the old mode instead: an independent emulated group per GPU.
 """
 from __future__ import annotations
 
@@ -181,16 +188,22 @@ class Clocks:
 
 # ---------------------------------------------------------------- helpers
 def setup_dist(args):
+    """(world, rank, device index).  One GPU per process over NCCL; with
+    --share-gpu every process uses GPU 0 over gloo (a correctness run of the
+    sharded path on one GPU: the processes time-share it)."""
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    local = 0 if args.share_gpu else int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
         import torch.distributed as dist
         torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        if args.share_gpu:
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=120))
+        else:
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
     else:
         torch.cuda.set_device(0)
     return world, rank, local
@@ -338,6 +351,27 @@ def run_ours(args, world, rank, local):
     with_ms = [e[0].elapsed_time(e[3]) for e in evs]
     without_ms = [e[0].elapsed_time(e[3]) for e in evs2]
 
+    # The launch floor of the planner in the same place of the step: a
+    # two-block plan (R=2, S=64, K=2, E=8) right after a full combine,
+    # between the same two events.  It is what an almost empty cooperative
+    # launch costs there; the planner's in-step time sits on top of it.
+    tk_t, _, _ = synth.routing(2, 64, 2, 8, 1.0, "boost0", seed=0)
+    h_t = moonep.moonep_create(64, 8, 2, 8, 2, 4, 8)
+    t_tk = torch.from_numpy(tk_t).to(dev)
+    p_t = moonep.Plan(h_t, dev)
+    floor = []
+    for i in range(max(8, min(args.steps, 20)) + 3):
+        moonep.moonep_combine(h, saved[i % npts], buf, wn, out, gw)
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        moonep.moonep_plan(h_t, t_tk, None, p_t)
+        a1.record(stream)
+        floor.append((a0, a1))
+    torch.cuda.synchronize()
+    plan_floor_us = statistics.median(a.elapsed_time(b) for a, b in floor[3:]) * 1e3
+    h_t.close()
+
     plan_ms = [e[0].elapsed_time(e[1]) for e in evs]
     disp_ms = [e[1].elapsed_time(e[2]) for e in evs]
     comb_ms = [e[2].elapsed_time(e[3]) for e in evs]
@@ -356,7 +390,7 @@ def run_ours(args, world, rank, local):
             realised_maxvio=round(r["realised"], 4),
             planner_us=round((statistics.median([with_ms[i] for i in idx]) -
                               statistics.median([without_ms[i] for i in idx])) * 1e3, 2),
-            planner_us_event_bracketed=round(statistics.mean([plan_ms[i] for i in idx]) * 1e3, 2),
+            planner_us_event_bracketed=round(statistics.median([plan_ms[i] for i in idx]) * 1e3, 2),
             dispatch_us=round(statistics.median([disp_ms[i] for i in idx]) * 1e3, 1),
             combine_us=round(statistics.median([comb_ms[i] for i in idx]) * 1e3, 1),
             dc_gbs=round(gbs, 1), dc_frac_measured=round(gbs / peak, 4), dc_frac_8tbs=round(gbs / NOMINAL_HBM_GBS, 4))
@@ -385,11 +419,13 @@ def run_ours(args, world, rank, local):
                    "step": "plan + dispatch + combine of one layer; combine reads the dispatch buffer"},
         # planner per layer: median step time with planning minus median
         # step time with saved plans, per routing, averaged over the sweep;
-        # also the planner between two CUDA events in each step (those come
-        # in ~2 us steps), and launched back to back alone
+        # also the median planner time between two CUDA events in each step
+        # (those come in ~2 us steps), launched back to back alone, and the
+        # in-step event time of a two-block planner launch (the launch floor)
         "planner_us": round(statistics.mean(v["planner_us"] for v in sweep.values()), 2),
-        "planner_us_event_bracketed": round(statistics.mean(plan_ms) * 1e3, 2),
+        "planner_us_event_bracketed": round(statistics.median(plan_ms) * 1e3, 2),
         "planner_us_back_to_back": round(plan_b2b_us, 2),
+        "planner_launch_floor_us": round(plan_floor_us, 2),
         "dispatch_gbs": round(db / (statistics.median(disp_ms) * 1e-3) / 1e9, 1),
         "combine_gbs": round(cb / (statistics.median(comb_ms) * 1e-3) / 1e9, 1),
         "dc_frac_measured_min": round(min(v["dc_frac_measured"] for v in sweep.values()), 4),
@@ -407,6 +443,7 @@ def run_ours(args, world, rank, local):
             result["legs"]["pages_maxvio_points"] = run_pages_points(w, seed, dev, h, plan, hidden, weights,
                                                                      buf, wn, out, gw, stream)
             result["legs"]["group_gemm"] = run_group_gemm_leg(dev, seed)
+            result["legs"]["fewest_copies"] = run_copies_leg(w, seed, dev)
             result["legs"]["rank_local"] = run_rank_local_leg(w, seed, dev, hidden, weights, routes, stream)
     if not args.no_e2e:
         result["e2e"] = run_e2e(args, h, plan, w, routes, dev, stream, world)
@@ -442,7 +479,7 @@ def run_pages_points(w, seed, dev, h, plan, hidden, weights, buf, wn, out, gw, s
         dc = statistics.median([e[1].elapsed_time(e[3]) for e in evs])
         pts[f"{mv:g}"] = dict(realised_maxvio=round(real, 4),
                               planner_us_event_bracketed=round(
-                                  statistics.mean([e[0].elapsed_time(e[1]) for e in evs]) * 1e3, 2),
+                                  statistics.median([e[0].elapsed_time(e[1]) for e in evs]) * 1e3, 2),
                               dispatch_us=round(statistics.median([e[1].elapsed_time(e[2]) for e in evs]) * 1e3, 1),
                               combine_us=round(statistics.median([e[2].elapsed_time(e[3]) for e in evs]) * 1e3, 1),
                               dc_gbs=round((db + cb) / (dc * 1e-3) / 1e9, 1),
@@ -536,6 +573,53 @@ def run_rank_local_leg(w, seed, dev, hidden, weights, routes, stream, reps=10):
                 timing="each phase's R launches as one CUDA graph, replayed between CUDA events; "
                        "'eager' = the same calls from Python",
                 points=res)
+
+
+def run_copies_leg(w, seed, dev, Hp=2048, n_proj=3, reps=50):
+    """Copies per layer of the two training planners on the same routings
+    (the sweep plus the pages' maxvio 10 and 20 points): used slots, i.e.
+    distinct (expert, recipient) pairs, and the weight bytes the prefetch of
+    those slots moves per layer (n_proj projections of [H, H'] bf16: each
+    distinct copied expert read once, each slot written once).  Mode 0 gives
+    a donor's experts away in id order, mode 3 largest first.  Also the
+    back-to-back planner time of each mode."""
+    import torch
+    from load_balancing_planner_b200 import moonep
+    R, S, K, E, B, H, tp = w["R"], w["S"], w["K"], w["E"], w["B"], w["H"], w["tp"]
+    hs = {m: moonep.moonep_create(S, H, K, E, R, B, tp, mode=m) for m in (0, 3)}
+    out = {"mv": [], "copies_mode0": [], "copies_mode3": [], "prefetch_gb_mode0": [], "prefetch_gb_mode3": []}
+    b2b = {}
+    routes = []
+    for mv in tuple(w["maxvio"]) + PAGES_POINTS:
+        tk, real, _ = synth.routing(R, S, K, E, mv, w["profile"], seed=seed)
+        routes.append((torch.from_numpy(tk).to(dev), torch.from_numpy(synth.local_counts(tk, E)).to(dev)))
+        out["mv"].append(mv)
+        for m, h in hs.items():
+            p = moonep.moonep_plan(h, *routes[-1])
+            torch.cuda.synchronize()
+            if moonep.moonep_read_status(p) != 0:
+                raise RuntimeError(f"mode {m} plan status")
+            se = p.slots().cpu().numpy()
+            U = int((se >= 0).sum())
+            D = int(np.unique(se[se >= 0]).size)
+            out[f"copies_mode{m}"].append(U)
+            out[f"prefetch_gb_mode{m}"].append(round(n_proj * (D + U) * H * Hp * 2 / 1e9, 2))
+    for m, h in hs.items():
+        p = moonep.Plan(h, dev)
+        for i in range(10):
+            moonep.moonep_plan(h, *routes[i % len(routes)], p)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        for i in range(reps):
+            moonep.moonep_plan(h, *routes[i % len(routes)], p)
+        b.record()
+        torch.cuda.synchronize()
+        b2b[f"mode{m}"] = round(a.elapsed_time(b) * 1e3 / reps, 2)
+        h.close()
+    out["planner_us_back_to_back"] = b2b
+    out["workload"] = f"{describe(w)}; prefetch of {n_proj} projections [H, H'={Hp}] bf16 per copy"
+    return out
 
 
 def run_group_gemm_leg(dev, seed, mv=2.0, Hp=2048, reps=10, config="train"):
@@ -738,6 +822,188 @@ def run_e2e(args, h, plan, w, routes, dev, stream, world):
             "pipelined": "uploads, compute and downloads of consecutive steps overlap on 3 streams"}
 
 
+# ---------------------------------------------------------------- EP over processes
+def ep_layout(R, world, rank):
+    """The EP ranks process `rank` of `world` owns: R/world consecutive ranks."""
+    if R % world:
+        raise ValueError(f"{R} EP ranks do not split over {world} processes")
+    per = R // world
+    return list(range(rank * per, (rank + 1) * per))
+
+
+def ep_bytes(R, S, K, H):
+    """Algorithmic bytes of one sharded layer: the same rows move as in the
+    emulated group (dispatch + combine of all R ranks' tokens)."""
+    return sum(dc_bytes(R, S, K, H))
+
+
+def run_ep(args, world, rank, local):
+    """One EP group of R ranks sharded over `world` processes (see the module
+    docstring).  Host barriers order the phases of every step: all plans
+    before any dispatch writes, all dispatches before any combine reads, all
+    combines before the next step's dispatch."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    from load_balancing_planner_b200 import ep, moonep
+
+    w = WORKLOADS[args.config]
+    R, S, K, E, B, H, tp = w["R"], w["S"], w["K"], w["E"], w["B"], w["H"], w["tp"]
+    mine = ep_layout(R, world, rank)
+    dev = torch.device("cuda", local)
+    nccl = dist.get_backend() == "nccl"
+    host = dist.new_group(backend="gloo", timeout=datetime.timedelta(seconds=120)) if nccl else None
+
+    # the whole group's routing from the shared seed; this process keeps its ranks' share
+    hid_all = synth.hidden_bf16(R, S, H, args.seed)
+    w_all = synth.route_weights(R, S, K, args.seed)
+    hidden = [hid_all[r].contiguous().to(dev) for r in mine]
+    weights = [torch.from_numpy(w_all[r].copy()).to(dev) for r in mine]
+    del hid_all
+    routes = []
+    for mv in w["maxvio"]:
+        tk, real, _ = synth.routing(R, S, K, E, mv, w["profile"], seed=args.seed)
+        tpe = synth.local_counts(tk, E)
+        routes.append(dict(target=mv, realised=real,
+                           topk=[torch.from_numpy(np.ascontiguousarray(tk[r])).to(dev) for r in mine],
+                           tpe=torch.from_numpy(tpe[mine].copy()).to(dev if nccl else "cpu")))
+    h = moonep.moonep_create(S, H, K, E, R, B, tp, mode=w["mode"])
+    nvs = h.nvs
+    bufs = [torch.empty((nvs, H), dtype=torch.bfloat16, device=dev) for _ in mine]
+    wbufs = [torch.empty((nvs,), dtype=torch.float32, device=dev) for _ in mine]
+    peers = ep.IpcPeers(bufs + wbufs, group=host)
+    per = len(mine)
+    # rank q's buffer: tensor (q % per) of process q // per
+    buf_tab = moonep.PeerTable([peers.rows[q // per][q % per] for q in range(R)], (nvs, H), torch.bfloat16)
+    w_tab = moonep.PeerTable([peers.rows[q // per][per + q % per] for q in range(R)], (nvs,), torch.float32)
+    plans = [moonep.Plan(h, dev, rank=r) for r in mine]
+    outs = [torch.empty((S, H), dtype=torch.bfloat16, device=dev) for _ in mine]
+    gws = [torch.empty((S, K), dtype=torch.float32, device=dev) for _ in mine]
+    stream = torch.cuda.current_stream(dev)
+    npts = len(routes)
+
+    def sync():
+        torch.cuda.synchronize(dev)
+        dist.barrier(group=host)
+
+    def gather(r):
+        # every rank's router counts, [R, E], in rank order
+        parts = [torch.empty_like(r["tpe"]) for _ in range(world)]
+        dist.all_gather(parts, r["tpe"])
+        return torch.cat(parts).to(dev)
+
+    def step(i, ev=None):
+        r = routes[i % npts]
+        if ev:
+            ev[0].record(stream)
+        counts = gather(r)
+        for j, q in enumerate(mine):
+            moonep.moonep_plan_rank(h, q, r["topk"][j], counts, plans[j])
+        sync()
+        if ev:
+            ev[1].record(stream)
+        for j in range(per):
+            moonep.moonep_dispatch_rank(h, plans[j], hidden[j], weights[j], buf_tab, w_tab)
+        sync()
+        if ev:
+            ev[2].record(stream)
+        for j in range(per):
+            moonep.moonep_combine_rank(h, plans[j], buf_tab, w_tab, outs[j], gws[j])
+        sync()
+        if ev:
+            ev[3].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+    sync()
+    st = max(moonep.moonep_read_status(p) for p in plans)
+    if st != 0:
+        raise RuntimeError(f"plan status {st}")
+    # the sharded step equals the emulated group's: each rank's plan against
+    # the group planner on the same routing, and the combined rows of the last
+    # step (weighted combine of the dispatched rows = the token itself)
+    check = moonep.moonep_plan(h, torch.from_numpy(synth.routing(R, S, K, E, w["maxvio"][(args.warmup - 1) % npts],
+                                                                 w["profile"], seed=args.seed)[0]).to(dev))
+    torch.cuda.synchronize(dev)
+    for j, q in enumerate(mine):
+        if not torch.equal(plans[j].dst, check.dst[q]):
+            raise RuntimeError(f"rank {q}: plan differs from the group plan")
+        if not torch.equal(outs[j].float(), hidden[j].float()):
+            raise RuntimeError(f"rank {q}: combine(dispatch(x)) is not x")
+    clocks = Clocks(local)
+    clocks.start()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    sync()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        step(i, evs[i])
+    t1.record(stream)
+    sync()
+    clk = clocks.stop()
+    total_ms = max_over_ranks(t0.elapsed_time(t1), world)
+    phase = [max_over_ranks(statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs), world) for j in range(3)]
+    total_b = ep_bytes(R, S, K, H)
+    value = total_b * args.steps / (total_ms * 1e-3) / 1e9
+    remote = sum(int((p.dst // nvs != q).sum().item()) for p, q in zip(plans, mine))
+    remote_rows = max_over_ranks(remote, world)
+
+    # e2e: every step also brings this process's ranks' inputs up from pinned
+    # host memory and takes their combined rows back down
+    hid_h = [x.cpu().pin_memory() for x in hidden]
+    w_h = [x.cpu().pin_memory() for x in weights]
+    tk_h = [[t.cpu().pin_memory() for t in r["topk"]] for r in routes]
+    out_h = [torch.empty((S, H), dtype=torch.bfloat16).pin_memory() for _ in mine]
+
+    def e2e_step(i):
+        r = routes[i % npts]
+        for j in range(per):
+            hidden[j].copy_(hid_h[j], non_blocking=True)
+            weights[j].copy_(w_h[j], non_blocking=True)
+            r["topk"][j].copy_(tk_h[i % npts][j], non_blocking=True)
+        step(i)
+        for j in range(per):
+            out_h[j].copy_(outs[j], non_blocking=True)
+        torch.cuda.synchronize(dev)
+
+    n_e2e = max(3, min(args.steps, 2 * npts))
+    e2e_step(0)
+    sync()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(n_e2e):
+        e2e_step(i)
+    b.record(stream)
+    sync()
+    e2e_ms = max_over_ranks(a.elapsed_time(b), world)
+    h2d = per * (S * H * 2 + S * K * 4 + S * K * 4)  # this process's hidden rows, route weights and picks
+    peers_n = world
+    peers.close()
+    h.close()
+    return {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4),
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": f"{args.config}: " + describe(w), "maxvio": list(w["maxvio"]),
+                   "parallelism": f"EP={R} sharded over {peers_n} processes, {per} ranks each; buffers mapped "
+                                  f"with CUDA IPC; phases ordered by host barriers",
+                   "l2": "inputs larger than L2",
+                   "step": "counts all-gather + plan_rank, dispatch_rank, combine_rank of every rank"},
+        "phase_ms_max_over_ranks": {"plan+gather": round(phase[0], 4), "dispatch": round(phase[1], 4),
+                                    "combine": round(phase[2], 4)},
+        "remote_picks_per_process_max": remote_rows,
+        "gpu_launches": 3 * per * args.steps,
+        "clocks": clk,
+        "e2e": {"value": round(total_b * n_e2e / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+                "h2d_bytes_per_step": int(h2d * world), "d2h_bytes_per_step": int(R * S * H * 2),
+                "ms_per_step": round(e2e_ms / n_e2e, 3), "steps": n_e2e},
+    }
+
+
 # ---------------------------------------------------------------- the oracle
 def oracle_sample(w, routes_np, ranks_sampled, seed):
     """Time the CPU oracle as it stands on one host core: the full plan of
@@ -886,6 +1152,9 @@ def split_result(result):
                                 for mv, v in pts.items()}
         evs = [v["plan_ev_us"] for v in line["sweep"].values()] + [v["plan_ev_us"] for v in line["pages_points"].values()]
         line["planner_us_event_bracketed_max"] = max(evs)
+    fc = detail.get("legs", {}).get("fewest_copies")
+    if fc:
+        line["copies_by_maxvio"] = {"mv": fc["mv"], "mode0": fc["copies_mode0"], "mode3": fc["copies_mode3"]}
     for k in ("prefetch_weight", "reduce_grad", "group_gemm"):
         leg = detail.get("legs", {}).get(k)
         if leg is None:
@@ -925,6 +1194,12 @@ def main():
                     help="time only the group GEMM on the workload (first maxvio of its sweep), for profiler "
                          "captures; prints the leg's JSON, not a bench line")
     ap.add_argument("--hp", type=int, default=2048, help="H' of the group GEMM")
+    ap.add_argument("--share-gpu", action="store_true",
+                    help="under torchrun: every process on GPU 0 over gloo (checks the sharded path on one GPU; "
+                         "its timings are not a measurement)")
+    ap.add_argument("--replicas", action="store_true",
+                    help="with --gpus N > 1: an independent emulated EP group per GPU instead of one group "
+                         "sharded over the GPUs")
     ap.add_argument("--planner-only", action="store_true",
                     help="launch only the planner (every routing of the workload), for profiler captures; "
                          "prints its back-to-back time, not a bench line")
@@ -950,6 +1225,14 @@ def main():
         return
 
     world, rank, local = setup_dist(args)
+    if world > 1 and not args.replicas:
+        result = run_ep(args, world, rank, local)
+        if rank == 0:
+            print(json.dumps(result), flush=True)
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+        return
     result, routes = run_ours(args, world, rank, local)
     if rank == 0 and world == 1 and not args.no_cpu:
         result["cpu_baseline"] = cpu_baseline(WORKLOADS[args.config], routes, args.seed)

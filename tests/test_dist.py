@@ -172,3 +172,15 @@ def test_bench_contract_line_is_short_and_keeps_the_headline_figures():
         assert k in line, k
     assert set(line["sweep"]) == set(sweep) and line["sweep"]["4"]["frac"] == 0.9144
     assert line["planner_us_event_bracketed_max"] == 19.9
+
+
+def test_ep_layout_splits_the_group_over_processes():
+    import bench
+    assert bench.ep_layout(8, 1, 0) == list(range(8))
+    assert bench.ep_layout(8, 2, 1) == [4, 5, 6, 7]
+    assert bench.ep_layout(8, 8, 3) == [3]
+    owned = sorted(q for p in range(4) for q in bench.ep_layout(8, 4, p))
+    assert owned == list(range(8))
+    with pytest.raises(ValueError):
+        bench.ep_layout(8, 3, 0)
+    assert bench.ep_bytes(8, 4096, 8, 7168) == sum(bench.dc_bytes(8, 4096, 8, 7168))
