@@ -344,12 +344,29 @@ def run_ours(args, world, rank, local):
 
     for i in range(args.warmup):
         step_saved(i)
-    evs2 = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    for i in range(args.steps):
-        step_saved(i, evs2[i])
+    # The planner's cost inside the step: the same steps with and without
+    # planning (the plans computed ahead), events only at the step
+    # boundaries, the two arms alternating, n_rep steps per routing and arm.
+    # The difference of the medians is what planning adds to a layer.
+    n_rep = 12
+    arms = {j: ([], []) for j in range(npts)}
+    for rep in range(n_rep + 1):
+        for j, r in enumerate(routes):
+            for arm in (0, 1):
+                a0 = torch.cuda.Event(enable_timing=True)
+                a1 = torch.cuda.Event(enable_timing=True)
+                a0.record(stream)
+                if arm == 0:
+                    moonep.moonep_plan(h, r["topk"], r["tpe"], plan)
+                p = plan if arm == 0 else saved[j]
+                moonep.moonep_dispatch(h, p, hidden, weights, buf, wn)
+                moonep.moonep_combine(h, p, buf, wn, out, gw)
+                a1.record(stream)
+                if rep:
+                    arms[j][arm].append((a0, a1))
     torch.cuda.synchronize()
-    with_ms = [e[0].elapsed_time(e[3]) for e in evs]
-    without_ms = [e[0].elapsed_time(e[3]) for e in evs2]
+    with_ms = {j: [a.elapsed_time(b) for a, b in v[0]] for j, v in arms.items()}
+    without_ms = {j: [a.elapsed_time(b) for a, b in v[1]] for j, v in arms.items()}
 
     # The launch floor of the planner in the same place of the step: a
     # two-block plan (R=2, S=64, K=2, E=8) right after a full combine,
@@ -388,8 +405,7 @@ def run_ours(args, world, rank, local):
         gbs = (db + cb) / (dc * 1e-3) / 1e9
         sweep[f"{r['target']:g}"] = dict(
             realised_maxvio=round(r["realised"], 4),
-            planner_us=round((statistics.median([with_ms[i] for i in idx]) -
-                              statistics.median([without_ms[i] for i in idx])) * 1e3, 2),
+            planner_us=round((statistics.median(with_ms[j]) - statistics.median(without_ms[j])) * 1e3, 2),
             planner_us_event_bracketed=round(statistics.median([plan_ms[i] for i in idx]) * 1e3, 2),
             dispatch_us=round(statistics.median([disp_ms[i] for i in idx]) * 1e3, 1),
             combine_us=round(statistics.median([comb_ms[i] for i in idx]) * 1e3, 1),
@@ -418,10 +434,12 @@ def run_ours(args, world, rank, local):
                    if args.config == "train" else "inputs larger than L2",
                    "step": "plan + dispatch + combine of one layer; combine reads the dispatch buffer"},
         # planner per layer: median step time with planning minus median
-        # step time with saved plans, per routing, averaged over the sweep;
+        # step time with saved plans (12 steps per routing and arm, events at
+        # the step boundaries only), per routing, averaged over the sweep;
         # also the median planner time between two CUDA events in each step
-        # (those come in ~2 us steps), launched back to back alone, and the
-        # in-step event time of a two-block planner launch (the launch floor)
+        # (those come in ~2 us steps and carry the gap an event pair opens
+        # between two kernels), launched back to back alone, and the in-step
+        # event time of a two-block planner launch (the launch floor)
         "planner_us": round(statistics.mean(v["planner_us"] for v in sweep.values()), 2),
         "planner_us_event_bracketed": round(statistics.median(plan_ms) * 1e3, 2),
         "planner_us_back_to_back": round(plan_b2b_us, 2),

@@ -300,6 +300,37 @@ __device__ __forceinline__ void alias_chain(int R, int C, const int *s_L, const 
     }
 }
 
+// Expert starts inside their group sequences in the fewest-copies order
+// (pick count ascending, ties by id): an expert starts after every expert of
+// its group that sorts before it.  Warps 1.. of the block; out of line, so
+// the kernel's own code is laid out the same in every mode.
+__device__ __noinline__ void expert_starts_by_count(const int32_t *T, int32_t *es, int E, int R, int G) {
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    if (G <= 32) {
+        // one warp per group, expert j on lane j: the counts go round the warp once
+        for (int h = w - 1; w >= 1 && h < R; h += kPlanWarps - 1) {
+            const int te = lane < G ? T[h * G + lane] : 0;
+            int sum = 0;
+#pragma unroll 1
+            for (int m = 0; m < 32; ++m) {
+                const int tm = __shfl_sync(0xffffffffu, te, m);
+                sum += (m < G && (tm < te || (tm == te && m < lane))) ? tm : 0;
+            }
+            if (lane < G) es[h * G + lane] = sum;
+        }
+    } else {
+        for (int e = tid - 32; w >= 1 && e < E; e += kPlanThreads - 32) {
+            const int g0 = e - e % G, te = T[e];
+            int sum = 0;
+            for (int m = g0; m < g0 + G; ++m) {
+                const int tm = T[m];
+                if (tm < te || (tm == te && m < e)) sum += tm;
+            }
+            es[e] = sum;
+        }
+    }
+}
+
 // ---- the planner kernel ----------------------------------------------------
 // 1024 threads per block: the register budget is 64 per thread.
 __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
@@ -637,30 +668,8 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
     // runs the alias chain).  Mode 3 (fewest copies) orders a group by pick
     // count, ties by id: an expert starts after every expert of its group
     // that sorts before it, one pass over the group per expert.
-    if (d.mode == 3 && G <= 32) {
-        // one warp per group, expert j on lane j: the group's counts are
-        // passed round the warp once
-        for (int h = w - 1; w >= 1 && h < R; h += kPlanWarps - 1) {
-            const int te = lane < G ? T[h * G + lane] : 0;
-            int sum = 0;
-            // not unrolled: this code runs once per block and is fetched cold
-#pragma unroll 1
-            for (int m = 0; m < 32; ++m) {
-                const int tm = __shfl_sync(0xffffffffu, te, m);
-                sum += (m < G && (tm < te || (tm == te && m < lane))) ? tm : 0;
-            }
-            if (lane < G) es[h * G + lane] = sum;
-        }
-    } else if (d.mode == 3) {
-        for (int e = tid - 32; w >= 1 && e < E; e += kPlanThreads - 32) {
-            const int g0 = e - e % G, te = T[e];
-            int sum = 0;
-            for (int m = g0; m < g0 + G; ++m) {
-                const int tm = T[m];
-                if (tm < te || (tm == te && m < e)) sum += tm;
-            }
-            es[e] = sum;
-        }
+    if (d.mode == 3) {
+        expert_starts_by_count(T, es, E, R, G);
     } else if (w >= 1) {
         for (int h = w - 1; h < R; h += kPlanWarps - 1) {
             int carry = 0;

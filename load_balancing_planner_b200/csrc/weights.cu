@@ -277,8 +277,12 @@ __global__ void __launch_bounds__(kWThreads) prefetch_bulk_kernel(const __grid_c
 #ifndef MOONEP_PF_RING
 #define MOONEP_PF_RING 4
 #endif
+#ifndef MOONEP_PF_INFLIGHT
+#define MOONEP_PF_INFLIGHT (MOONEP_PF_RING / 2)
+#endif
 constexpr int kPfRing = MOONEP_PF_RING;
-constexpr int kPfInFlight = kPfRing / 2;
+constexpr int kPfInFlight = MOONEP_PF_INFLIGHT;
+static_assert(kPfInFlight >= 1 && kPfInFlight < kPfRing, "stores in flight must leave a stage for loads");
 
 __global__ void __launch_bounds__(kWThreads) prefetch_ring_kernel(const __grid_constant__ WeightArgs a) {
     __shared__ volatile int s_abort;
@@ -435,7 +439,13 @@ __global__ void __launch_bounds__(kWThreads) reduce_grad_kernel(const __grid_con
 // completing on mbarriers); the other 8 warps add them up in registers (16
 // floats a thread), in that order, store the sum to the grad and zeros to
 // the holders, and hand each ring slot back as soon as they have read it.
-constexpr int kRgRing = 6;
+#ifndef MOONEP_RG_RING
+#define MOONEP_RG_RING 6
+#endif
+#ifndef MOONEP_RG_BPS
+#define MOONEP_RG_BPS 2
+#endif
+constexpr int kRgRing = MOONEP_RG_RING;
 constexpr int kRgTile = 4096;                  // floats per piece (16 KB)
 constexpr int kRgThreads = 32 + 256;           // producer warp + 8 summing warps
 constexpr int kRgPer = kRgTile / 256;          // floats per summing thread
@@ -638,13 +648,13 @@ bool reduce_grad_use_bulk(const WeightArgs &a) {
     for (int p = 0; p < a.n_proj; ++p)
         aligned = aligned && (reinterpret_cast<uintptr_t>(a.src[p]) % 16) == 0 &&
                   (reinterpret_cast<uintptr_t>(a.dst[p]) % 16) == 0;
-    return aligned && a.hhp >= kRgTile && reduce_bulk_smem(a) <= 110 * 1024;
+    return aligned && a.hhp >= kRgTile && reduce_bulk_smem(a) <= (MOONEP_RG_BPS == 1 ? 220 : 110) * 1024;
 }
 
 cudaError_t launch_reduce_grad(const WeightArgs &a, int grid, int sms, cudaStream_t st) {
     if (a.remote || !reduce_grad_use_bulk(a)) return launch_w(reduce_grad_kernel, a, grid, st);
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(2 * sms));  // two rings per SM
+    cfg.gridDim = dim3((unsigned)(MOONEP_RG_BPS * sms));  // rings per SM
     cfg.blockDim = dim3(kRgThreads);
     cfg.dynamicSmemBytes = reduce_bulk_smem(a);
     cfg.stream = st;
