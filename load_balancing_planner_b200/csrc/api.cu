@@ -155,9 +155,11 @@ int plan_dims(const moonep_config_t &cfg, int device, Dims *out, int *grid) {
     d.ct = d.S < kChunkTokensMin ? d.S : kChunkTokensMin;
     for (int iter = 0; iter < 8; ++iter) {
         d.nch = (d.S + d.ct - 1) / d.ct;
-        // second-recipient bases only where the layout tables still fit
+        // the optional layout tables only where they still fit
         d.cw = 1;
         d.fast2 = 1;
+        d.xtab = 1;
+        if (plan_smem_bytes(d) > smem_max) d.xtab = 0;
         if (plan_smem_bytes(d) > smem_max) d.fast2 = 0;
         d.cw = kPlanWarps;
         while (d.cw > 1 && plan_smem_bytes(d) > smem_max) d.cw /= 2;

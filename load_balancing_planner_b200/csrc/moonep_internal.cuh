@@ -26,6 +26,7 @@ struct Dims {
     int NR;   // rows per rank = E + B
     int nvs;  // NvS
     int fast2;  // planner keeps second-recipient dst bases (when shared memory allows)
+    int xtab;   // planner keeps the split column pass's and the rank pass's dst-base tables (when they fit)
 };
 
 // Planning workspace (one device allocation owned by the handle).

@@ -32,6 +32,13 @@
 // every block validates first, and the alias chain follows the column pass.
 #include "moonep_internal.cuh"
 
+#ifndef MOONEP_PLAN_COLSPLIT
+#define MOONEP_PLAN_COLSPLIT 1
+#endif
+#ifndef MOONEP_PLAN_FOLDRANK
+#define MOONEP_PLAN_FOLDRANK 1
+#endif
+
 namespace moonep {
 
 __host__ __device__ static inline size_t align256(size_t b) { return (b + 255) / 256 * 256; }
@@ -63,9 +70,9 @@ __host__ __device__ static size_t region1_bytes(const Dims &d) {
     // counting phase: per-warp counts + per-warp lane masks; layout phase reuses it
     const size_t counts = counts_bytes(d) + sizeof(uint32_t) * (size_t)d.cw * d.E;
     // int32: T, pre, es, nhome, kbase, nrecv, ovfincl, recvstart, ebase, eend
-    // (10 E), ebase2, eend2 (2 E, when fast2) + slotincl (R B);
-    // int16: qidx (E) + slotj (R B)
-    const size_t layout = sizeof(int32_t) * ((10 + 2 * (size_t)d.fast2) * d.E + (size_t)d.R * d.B) +
+    // (10 E), ebase2, eend2 (2 E, when fast2) + slotincl (R B) + pre2, dbase,
+    // dlim (3 E, when xtab); int16: qidx (E) + slotj (R B)
+    const size_t layout = sizeof(int32_t) * ((10 + 2 * (size_t)d.fast2 + 3 * (size_t)d.xtab) * d.E + (size_t)d.R * d.B) +
                           sizeof(int16_t) * ((size_t)d.E + (size_t)d.R * d.B + 2);
     return align256(counts > layout ? counts : layout);
 }
@@ -509,7 +516,16 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
     int32_t *ebase2 = eend + E;         // [E] the same for the second recipient (fast2 only)
     int32_t *eend2 = ebase2 + E;        // [E]
     int32_t *slotincl = eend + E + (d.fast2 ? 2 * E : 0);  // [R*B] inclusive padded running sum over the slot rows
-    int16_t *qidx = reinterpret_cast<int16_t *>(slotincl + R * B);  // [R*G] received-expert index, -1 none
+    // [E] picks of e in this rank's earlier chunks, when the column pass
+    // sums those rows on warps of their own (pre then holds only the picks
+    // of earlier ranks)
+    int32_t *pre2 = slotincl + R * B;
+    // [E] the dst base of a kept pick of e relative to this chunk, and the
+    // chunk rank below which picks of e are kept (set in the rank pass)
+    int32_t *dbase = pre2 + E;
+    int32_t *dlim = dbase + E;
+    // (pre2, dbase and dlim exist when the layout tables have room: d.xtab)
+    int16_t *qidx = reinterpret_cast<int16_t *>(slotincl + R * B + (d.xtab ? 3 * E : 0));  // [R*G] received-expert index, -1 none
     int16_t *slotj = qidx + E;          // [R*B] donor-group index of the expert in slot b
 
     __shared__ int s_L[MOONEP_MAX_R], s_keep[MOONEP_MAX_R];
@@ -524,6 +540,11 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
     // chain while the others do the column pass.  One rank's planning gets
     // its loads from the column pass below.
     const int aw = min(kPlanWarps - 1, (E + 31) / 32);
+    // the split column pass: experts on threads [0, E) and again on the
+    // threads after the alias warp, [col2, col2 + E)
+    const int col2 = 32 * (aw + 1);
+    const bool colsplit = MOONEP_PLAN_COLSPLIT && d.xtab && col2 + E <= kPlanThreads;
+    const bool foldrank = MOONEP_PLAN_FOLDRANK && d.xtab;
     if (!one_rank && w == aw) {
         for (int h = lane; h < R; h += 32) s_L[h] = ld_cg(a.ws.gload + (size_t)parity * R + h);
         __syncwarp();
@@ -550,20 +571,21 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
         // rows q < R are the per-rank counts, rows R <= q < R + c this rank's
         // earlier chunk histograms; 16 loads in flight per batch
         const int nrows = R + c;
-        for (int e = tid; e < E; e += kPlanThreads) {
-            int tot = 0, mypre = 0, myv = 0;
-            for (int q0 = 0; q0 < nrows; q0 += 16) {
-                int v[16];
+        if (colsplit) {
+            // warps 0.. sum the per-rank counts, the warps after the alias
+            // warp this rank's earlier chunk rows: one batch of loads each
+            // for up to 16 rows, where one thread per expert took two
+            if (tid < E) {
+                const int e = tid;
+                int tot = 0, mypre = 0, myv = 0;
+                for (int q0 = 0; q0 < R; q0 += 16) {
+                    int v[16];
 #pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    const int q = q0 + u;
-                    const int32_t *src = q < R ? cnt + (int64_t)q * E + e : mine_rows + (int64_t)(q - R) * E + e;
-                    v[u] = q < nrows ? ld_cg(src) : 0;
-                }
+                    for (int u = 0; u < 16; ++u) v[u] = q0 + u < R ? ld_cg(cnt + (int64_t)(q0 + u) * E + e) : 0;
 #pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    const int q = q0 + u;
-                    if (q < R) {
+                    for (int u = 0; u < 16; ++u) {
+                        const int q = q0 + u;
+                        if (q >= R) continue;
                         tot += v[u];
                         if (q < r) mypre += v[u];
                         if (q == r) myv = v[u];
@@ -571,15 +593,56 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
                             const int t = tpe_in_smem(d) ? tpe_s[q * E + e] : __ldg(a.tpe + (int64_t)q * E + e);
                             if (t != v[u]) mismatch = true;
                         }
-                    } else {
-                        mypre += v[u];  // 0 past the last row
                     }
                 }
+                T[e] = tot;
+                pre[e] = mypre;
+                if (c == 0 && !one_rank) a.plan.counts[(int64_t)r * E + e] = myv;
+                if (checker && one_rank && ld_cg(own + e) != myv) mismatch = true;  // the rank's own row
+            } else if (tid >= col2 && tid < col2 + E) {
+                const int e = tid - col2;
+                int sum = 0;
+                for (int q0 = 0; q0 < c; q0 += 16) {
+                    int v[16];
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) v[u] = q0 + u < c ? ld_cg(mine_rows + (int64_t)(q0 + u) * E + e) : 0;
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) sum += v[u];
+                }
+                pre2[e] = sum;
             }
-            T[e] = tot;
-            pre[e] = mypre;
-            if (c == 0 && !one_rank) a.plan.counts[(int64_t)r * E + e] = myv;
-            if (checker && one_rank && ld_cg(own + e) != myv) mismatch = true;  // the rank's own row
+        } else {
+            for (int e = tid; e < E; e += kPlanThreads) {
+                int tot = 0, mypre = 0, myv = 0;
+                for (int q0 = 0; q0 < nrows; q0 += 16) {
+                    int v[16];
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) {
+                        const int q = q0 + u;
+                        const int32_t *src = q < R ? cnt + (int64_t)q * E + e : mine_rows + (int64_t)(q - R) * E + e;
+                        v[u] = q < nrows ? ld_cg(src) : 0;
+                    }
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) {
+                        const int q = q0 + u;
+                        if (q < R) {
+                            tot += v[u];
+                            if (q < r) mypre += v[u];
+                            if (q == r) myv = v[u];
+                            if (checker && !one_rank) {
+                                const int t = tpe_in_smem(d) ? tpe_s[q * E + e] : __ldg(a.tpe + (int64_t)q * E + e);
+                                if (t != v[u]) mismatch = true;
+                            }
+                        } else {
+                            mypre += v[u];  // 0 past the last row
+                        }
+                    }
+                }
+                T[e] = tot;
+                pre[e] = mypre;
+                if (c == 0 && !one_rank) a.plan.counts[(int64_t)r * E + e] = myv;
+                if (checker && one_rank && ld_cg(own + e) != myv) mismatch = true;  // the rank's own row
+            }
         }
     }
     // the router's counts are checked by block 0 only, which writes the
@@ -776,6 +839,14 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
         for (int j = lane; j < G; j += 32) {
             const int e = s * G + j;
             kbase[e] = s * d.nvs + off_home + kbase[e] - pad_to(nhome[e], tp) - es[e];
+            if (foldrank) {
+                // this block's offset of e (its start in the group sequence
+                // plus the picks of earlier ranks and chunks): a kept pick of
+                // chunk rank rk goes to dbase[e] + rk while rk < dlim[e]
+                const int off = es[e] + pre[e] + (colsplit ? pre2[e] : 0);
+                dbase[e] = kbase[e] + off;
+                dlim[e] = keep_s - off;
+            }
             if (h >= 0) {
                 const int q = qidx[s * G + j];
                 const int p = pad_to(nrecv[s * G + j], tp);
@@ -789,7 +860,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
                 // relative to this block's chunk: a pick of chunk rank rk
                 // sits at g = off + rk in the group sequence.
                 const int eh = h * G + j;
-                const int off = es[eh] + pre[eh];
+                const int off = es[eh] + pre[eh] + (colsplit ? pre2[eh] : 0);
                 const int lo = max(es[eh], s_keep[h]);
                 const int a0 = s_rstart[s], a1 = a0 + s_rlen[s];
                 if (q >= 0 && a0 <= lo && lo < a1) {
@@ -873,32 +944,37 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
         PLAN_TRACE(13);
     } else {
         const int t2 = tid - 32 * ow, n2 = kPlanThreads - 32 * ow;
-        // Fold this block's offset of each expert (its start in the group
-        // sequence plus the picks of earlier chunks) into the kept-pick base
-        // and limit, so a pick of rank rk inside the chunk needs only rk: its
-        // position in the group sequence is g = off + rk.  The outputs never
-        // read the arrays rewritten here (T, pre).
-        for (int e = t2; e < E; e += n2) {
-            const int off = es[e] + pre[e];
-            T[e] = kbase[e] + off;           // kept pick: dst = T[e] + rk ...
-            pre[e] = s_keep[e / G] - off;    // ... while rk < pre[e]
+        int32_t *kb = dbase, *kl = dlim;
+        if (!foldrank) {
+            // Fold this block's offset of each expert (its start in the group
+            // sequence plus the picks of earlier chunks) into the kept-pick
+            // base and limit, so a pick of rank rk inside the chunk needs only
+            // rk: its position in the group sequence is g = off + rk.  The
+            // outputs never read the arrays rewritten here (T, pre).
+            for (int e = t2; e < E; e += n2) {
+                const int off = es[e] + pre[e] + (colsplit ? pre2[e] : 0);
+                T[e] = kbase[e] + off;           // kept pick: dst = T[e] + rk ...
+                pre[e] = s_keep[e / G] - off;    // ... while rk < pre[e]
+            }
+            asm volatile("bar.sync 1, %0;" ::"r"(n2) : "memory");
+            kb = T;
+            kl = pre;
         }
-        asm volatile("bar.sync 1, %0;" ::"r"(n2) : "memory");
         PLAN_TRACE_BY(12, 32 * ow);
         // destination of every pick of this block's chunk
         for (int i = t2; i < n_ent; i += n2) {
             const int e = ent_e[i];
             const int rk = ent_rank[i];
             int dst;
-            if (rk < pre[e]) {
-                dst = T[e] + rk;
+            if (rk < kl[e]) {
+                dst = kb[e] + rk;
             } else if (rk < eend[e]) {
                 dst = ebase[e] + rk;
             } else if (d.fast2 && rk < eend2[e]) {
                 dst = ebase2[e] + rk;
             } else {  // the expert's donated run spans three or more recipients
                 const int h = e / G;
-                const int g = rk + s_keep[h] - pre[e];
+                const int g = rk + s_keep[h] - kl[e];
                 int dest = -1;
                 for (int k = s_doff[h]; k < s_doff[h + 1]; ++k) {
                     const int s = s_dlist[k];
