@@ -426,10 +426,11 @@ def run_ours(args, world, rank, local):
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms_max / args.steps, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic",
+        "higher_is_better": True, "scaling": "weak" if args.replicas else "strong", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
         "config": {"workload": f"{args.config}: " + describe(w), "maxvio": list(w["maxvio"]),
-                   "parallelism": f"EP={R} emulated on each GPU; independent EP groups per GPU",
+                   "parallelism": (f"EP={R} emulated on each GPU; independent EP groups per GPU" if args.replicas
+                                   else f"EP={R} emulated on one GPU (--gpus N shards the same group over N GPUs)"),
                    "l2": "inputs larger than L2 (hidden rows 470 MB, dispatch buffer 4.7 GB per layer)"
                    if args.config == "train" else "inputs larger than L2",
                    "step": "plan + dispatch + combine of one layer; combine reads the dispatch buffer"},
@@ -1112,7 +1113,7 @@ def run_reference(args, world, rank):
     return {
         "impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ts / args.steps * 1e3, 1),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
         "config": {"workload": f"{args.config}: " + describe(w), "maxvio": list(w["maxvio"])},
         "cpu_baseline": {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle",

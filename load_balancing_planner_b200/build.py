@@ -41,7 +41,12 @@ def _stale() -> bool:
     return any(os.path.getmtime(f) > t for f in deps)
 
 
+last_build_compiled = False  # whether the last build() call ran nvcc
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
+    global last_build_compiled
+    last_build_compiled = False
     if not force and not _stale():
         return LIB
     tmp = LIB + f".tmp{os.getpid()}"
@@ -50,6 +55,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
         print(" ".join(cmd), flush=True)
     subprocess.run(cmd, check=True)
     os.replace(tmp, LIB)
+    last_build_compiled = True
     return LIB
 
 

@@ -197,7 +197,10 @@ __global__ void __launch_bounds__(kWThreads) prefetch_kernel(const __grid_consta
 // bulk store per slot holding the expert, and the stage is refilled as soon
 // as those stores have read it.  Every expert piece is read once.
 constexpr int kPfStages = 3;
-constexpr uint32_t kPfTile = 32 * 1024;
+#ifndef MOONEP_PF_TILE_KB
+#define MOONEP_PF_TILE_KB 32
+#endif
+constexpr uint32_t kPfTile = MOONEP_PF_TILE_KB * 1024;
 
 __global__ void __launch_bounds__(kWThreads) prefetch_bulk_kernel(const __grid_constant__ WeightArgs a) {
     pdl_wait();
@@ -593,15 +596,18 @@ static size_t prefetch_bulk_smem(const WeightArgs &a) {
     return ((weights_smem(a) + 127) & ~(size_t)127) + kPfStages * (size_t)kPfTile + 8 * kPfStages;
 }
 
-// The bulk prefetch needs 16-byte aligned matrices of whole 16-byte units and
-// room for its ring next to the slot tables.
-bool prefetch_use_bulk(const WeightArgs &a) {
+// The bulk prefetch kernels need 16-byte aligned matrices of whole 16-byte
+// units, at least one piece long.
+static bool prefetch_bulk_fits(const WeightArgs &a) {
     bool aligned = ((a.hhp * 2) % 16) == 0;
     for (int p = 0; p < a.n_proj; ++p)
         aligned = aligned && (reinterpret_cast<uintptr_t>(a.src[p]) % 16) == 0 &&
                   (reinterpret_cast<uintptr_t>(a.dst[p]) % 16) == 0;
-    return aligned && a.hhp * 2 >= kPfTile && prefetch_bulk_smem(a) <= 110 * 1024;
+    return aligned && a.hhp * 2 >= kPfTile;
 }
+
+// ... and the older kernel room for its ring next to the slot tables
+bool prefetch_use_bulk(const WeightArgs &a) { return prefetch_bulk_fits(a) && prefetch_bulk_smem(a) <= 110 * 1024; }
 
 static size_t prefetch_ring_smem(const WeightArgs &a) {
     return ((weights_smem(a) + 127) & ~(size_t)127) + kPfRing * (size_t)kPfTile + 16 * kPfRing;
@@ -612,7 +618,7 @@ static size_t prefetch_ring_smem(const WeightArgs &a) {
 #endif
 
 cudaError_t launch_prefetch(const WeightArgs &a, int grid, int sms, cudaStream_t st) {
-    if (a.remote || !prefetch_use_bulk(a)) return launch_w(prefetch_kernel, a, grid, st);
+    if (a.remote || !prefetch_bulk_fits(a)) return launch_w(prefetch_kernel, a, grid, st);
     if (MOONEP_PF_USE_RING && prefetch_ring_smem(a) <= 220 * 1024) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)sms);  // one deep ring per SM
@@ -626,6 +632,7 @@ cudaError_t launch_prefetch(const WeightArgs &a, int grid, int sms, cudaStream_t
         cfg.numAttrs = 1;
         return cudaLaunchKernelEx(&cfg, prefetch_ring_kernel, a);
     }
+    if (!prefetch_use_bulk(a)) return launch_w(prefetch_kernel, a, grid, st);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(2 * sms));  // two rings per SM
     cfg.blockDim = dim3(kWThreads);
