@@ -29,6 +29,7 @@ CASES = [
     ("tiny", 2, 64, 2, 8, 4, 128, 8, 0, "boost0", 1.0, 16),
     ("bulk_rows", 4, 512, 4, 32, 8, 1024, 16, 0, "hot8", 2.0, 64),
     ("infer_overflow", 3, 300, 3, 24, 2, 264, 16, 1, "hot8", 3.0, 24),
+    ("fewest_copies", 4, 512, 4, 32, 8, 1024, 16, 3, "hot8", 2.0, 64),
 ]
 
 
@@ -182,24 +183,25 @@ def test_one_rank_per_process_matches_the_oracle(cuda, case):
         assert p.exitcode == 0
 
 
-def test_bench_sharded_ep_mode_on_one_gpu(cuda):
-    # `bench.py --gpus 2` in its sharded mode, with both processes on this
-    # GPU (--share-gpu, gloo): each process owns 4 of the 8 EP ranks, maps the
-    # other's buffers with CUDA IPC, and checks its plans against the group
+@pytest.mark.parametrize("nproc", [2, 4])
+def test_bench_sharded_ep_mode_on_one_gpu(cuda, nproc):
+    # `bench.py --gpus N` in its sharded mode, with every process on this GPU
+    # (--share-gpu, gloo): each process owns 8/N of the 8 EP ranks, maps the
+    # others' buffers with CUDA IPC, and checks its plans against the group
     # planner and combine(dispatch(x)) = x before timing; one contract line
     import json
     import subprocess
     import sys
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
-           "--master-addr", "127.0.0.1", "--master-port", str(_free_port()), "bench.py", "--gpus", "2",
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", str(nproc),
+           "--master-addr", "127.0.0.1", "--master-port", str(_free_port()), "bench.py", "--gpus", str(nproc),
            "--share-gpu", "--config", "zipf", "--steps", "3", "--warmup", "3"]
     out = subprocess.run(cmd, cwd=root, capture_output=True, text=True, timeout=900)
     assert out.returncode == 0, (out.stdout[-2000:], out.stderr[-3000:])
     lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
     assert len(lines) == 1, out.stdout[-2000:]
     d = json.loads(lines[0])
-    assert d["n_gpus"] == 2 and d["scaling"] == "strong" and d["value"] > 0
-    assert "EP=8 sharded over 2 processes" in d["config"]["parallelism"]
+    assert d["n_gpus"] == nproc and d["scaling"] == "strong" and d["value"] > 0
+    assert f"EP=8 sharded over {nproc} processes, {8 // nproc} ranks each" in d["config"]["parallelism"]
     assert d["remote_picks_per_process_max"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] > 0
