@@ -348,7 +348,7 @@ def run_ours(args, world, rank, local):
     # planning (the plans computed ahead), events only at the step
     # boundaries, the two arms alternating, n_rep steps per routing and arm.
     # The difference of the medians is what planning adds to a layer.
-    n_rep = 12
+    n_rep = 24
     arms = {j: ([], []) for j in range(npts)}
     for rep in range(n_rep + 1):
         for j, r in enumerate(routes):
@@ -435,7 +435,7 @@ def run_ours(args, world, rank, local):
                    if args.config == "train" else "inputs larger than L2",
                    "step": "plan + dispatch + combine of one layer; combine reads the dispatch buffer"},
         # planner per layer: median step time with planning minus median
-        # step time with saved plans (12 steps per routing and arm, events at
+        # step time with saved plans (24 steps per routing and arm, events at
         # the step boundaries only), per routing, averaged over the sweep;
         # also the median planner time between two CUDA events in each step
         # (those come in ~2 us steps and carry the gap an event pair opens
