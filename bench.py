@@ -682,16 +682,16 @@ def run_group_gemm_leg(dev, seed, mv=2.0, Hp=2048, reps=10, config="train"):
             "peak_kind": kind, "rows_real": R * S * K, "rows_computed": rows_computed}
 
 
-def run_legs(args, dev, world):
+def run_legs(args, dev, world, Hp=2048, reps=5):
     """prefetch_weight at the inference shape and reduce_grad at the backward
-    shape, timed with CUDA events (median of reps)."""
+    shape, timed with CUDA events (median of reps).  A smaller H' gives the
+    same kernels on less memory, for profiler captures."""
     import torch
     from load_balancing_planner_b200 import moonep
     legs = {}
     peak, _ = peaks()
-    R, S, K, E, H, Hp, tp = 8, 4096, 8, 256, 7168, 2048, 128
+    R, S, K, E, H, tp = 8, 4096, 8, 256, 7168, 128
     gen = torch.Generator(device=dev).manual_seed(args.seed)
-    reps = 5
 
     def timed(fn):
         ts = []
@@ -733,7 +733,7 @@ def run_legs(args, dev, world):
                               us=round(ms * 1e3, 1), gbs=round(by / (ms * 1e-3) / 1e9, 1),
                               frac_measured=round(by / (ms * 1e-3) / 1e9 / peak, 4),
                               overflow_picks_slots_by_id=ovf[1], overflow_picks_slots_by_count=ovf[2])
-    legs["prefetch_weight"] = dict(workload="inference R=8 S=4096 K=8 E=256 B=4 H=7168 H'=2048, 3 projections",
+    legs["prefetch_weight"] = dict(workload=f"inference R=8 S=4096 K=8 E=256 B=4 H=7168 H'={Hp}, 3 projections",
                                    bytes="3*(D+U)*H*H'*2", points=out)
     del Ws, pools
     h.close()
@@ -750,7 +750,7 @@ def run_legs(args, dev, world):
     D = int(np.unique(se[se >= 0]).size)
     ms = timed(lambda: moonep.moonep_reduce_grad(h, p, [G], [RB]))
     by = (2 * D + 2 * U) * H * Hp * 4
-    legs["reduce_grad"] = dict(workload="backward E=256 R=8 B=32 H=7168 H'=2048 fp32, plan at maxvio 2",
+    legs["reduce_grad"] = dict(workload=f"backward E=256 R=8 B=32 H=7168 H'={Hp} fp32, plan at maxvio 2",
                                bytes="(2D+2U)*H*H'*4", realised_maxvio=round(real, 4), used_slots=U,
                                distinct_experts=D, us=round(ms * 1e3, 1),
                                gbs=round(by / (ms * 1e-3) / 1e9, 1),
@@ -1212,7 +1212,10 @@ def main():
     ap.add_argument("--gemm-only", action="store_true",
                     help="time only the group GEMM on the workload (first maxvio of its sweep), for profiler "
                          "captures; prints the leg's JSON, not a bench line")
-    ap.add_argument("--hp", type=int, default=2048, help="H' of the group GEMM")
+    ap.add_argument("--hp", type=int, default=2048, help="H' of the group GEMM and of the weight legs")
+    ap.add_argument("--weights-only", action="store_true",
+                    help="run only the prefetch_weight and reduce_grad legs at H' = --hp, --steps timed launches "
+                         "per point, for profiler captures; prints the legs' JSON, not a bench line")
     ap.add_argument("--share-gpu", action="store_true",
                     help="under torchrun: every process on GPU 0 over gloo (checks the sharded path on one GPU; "
                          "its timings are not a measurement)")
@@ -1227,6 +1230,10 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.planner_only:
         print(json.dumps(run_planner_only(args)), flush=True)
+        return
+    if args.weights_only:
+        import torch
+        print(json.dumps(run_legs(args, torch.device("cuda", 0), 1, Hp=args.hp, reps=args.steps)), flush=True)
         return
     if args.gemm_only:
         import torch
