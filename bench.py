@@ -694,16 +694,17 @@ def run_legs(args, dev, world, Hp=2048, reps=5):
     gen = torch.Generator(device=dev).manual_seed(args.seed)
 
     def timed(fn):
-        ts = []
-        for _ in range(reps + 1):
-            a = torch.cuda.Event(enable_timing=True)
-            b = torch.cuda.Event(enable_timing=True)
+        # All launches are enqueued back to back, so each start event is
+        # reached while the launch before it runs and the launch itself is
+        # already queued: the events time the kernel, not the host's launch
+        # latency.  The first pair starts on an idle stream and is dropped.
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps + 1)]
+        for a, b in evs:
             a.record()
             fn()
             b.record()
-            torch.cuda.synchronize()
-            ts.append(a.elapsed_time(b))
-        return statistics.median(ts[1:])
+        torch.cuda.synchronize()
+        return statistics.median(a.elapsed_time(b) for a, b in evs[1:])
 
     # prefetch_weight: inference, B = 4, three projections
     h = moonep.moonep_create(S, H, K, E, R, 4, tp, mode=1)

@@ -180,9 +180,11 @@ struct AliasOut {
 };
 
 // The balancing assignment in closed form, run by one warp: rank h lives on
-// lane h % 32, slot h / 32 (NS slots cover R <= 32 * NS ranks).
+// lane h % 32, slot h / 32 (NS slots cover R <= 32 * NS ranks).  Out of line:
+// its call sites (group and one-rank planning, both rank-slot counts) share
+// one copy of the code.
 template <int NS>
-__device__ __forceinline__ void alias_chain(int R, int C, const int *s_L, const AliasOut &o) {
+__device__ __noinline__ void alias_chain(int R, int C, const int *s_L, const AliasOut o) {
     const int lane = threadIdx.x & 31;
     int Lv[NS], D[NS], X[NS], Pin[NS], Qin[NS], Pex[NS], Qex[NS];
     int carryP = 0, carryQ = 0;
@@ -338,9 +340,158 @@ __device__ __noinline__ void expert_starts_by_count(const int32_t *T, int32_t *e
     }
 }
 
+// The helpers below hold paths that the common configurations never take (or
+// take on a few threads), kept out of line with the alias chain: the planner
+// is latency-bound, its warps fetch their code cold after the streaming
+// kernels of a layer, and every cache line of code on the way costs time, so
+// the kernel's own path stays compact.
+
+// Duplicate picks token by token, for K that does not divide 32 (a token's
+// picks then straddle the counting warps' runs of 32).  Out of line: the
+// common K keep it off the kernel's own code path.
+__device__ __noinline__ int dup_by_token(const uint16_t *ent_e, int ntok, int K) {
+    int bad = 0;
+    for (int tt = threadIdx.x; tt < ntok; tt += kPlanThreads) {
+        const uint16_t *tok = ent_e + tt * K;
+        for (int k = 1; k < K; ++k) {
+            const uint16_t ek = tok[k];
+            if (ek == 0xFFFF) continue;
+            for (int k2 = 0; k2 < k; ++k2)
+                if (tok[k2] == ek) bad |= MOONEP_STATUS_DUP_EXPERT;
+        }
+    }
+    return bad;
+}
+
+// The column pass in one loop per expert (rows of the per-rank counts, then
+// this rank's earlier chunk rows), for configurations whose layout tables
+// leave no room for the split form.  Returns this thread's count mismatch.
+__device__ __noinline__ bool column_pass_one_loop(const PlanArgs &a, const int32_t *cnt, const int32_t *own,
+                                                  const int32_t *mine_rows, const int32_t *tpe_s, int32_t *T,
+                                                  int32_t *pre, int r, int c, bool checker, bool one_rank) {
+    const Dims &d = a.d;
+    const int E = d.E, R = d.R, nrows = R + c;
+    bool mismatch = false;
+    for (int e = threadIdx.x; e < E; e += kPlanThreads) {
+        int tot = 0, mypre = 0, myv = 0;
+        for (int q0 = 0; q0 < nrows; q0 += 16) {
+            int v[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const int q = q0 + u;
+                const int32_t *src = q < R ? cnt + (int64_t)q * E + e : mine_rows + (int64_t)(q - R) * E + e;
+                v[u] = q < nrows ? ld_cg(src) : 0;
+            }
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const int q = q0 + u;
+                if (q < R) {
+                    tot += v[u];
+                    if (q < r) mypre += v[u];
+                    if (q == r) myv = v[u];
+                    if (checker && !one_rank) {
+                        const int t = tpe_in_smem(d) ? tpe_s[q * E + e] : __ldg(a.tpe + (int64_t)q * E + e);
+                        if (t != v[u]) mismatch = true;
+                    }
+                } else {
+                    mypre += v[u];  // 0 past the last row
+                }
+            }
+        }
+        T[e] = tot;
+        pre[e] = mypre;
+        if (c == 0 && !one_rank) a.plan.counts[(int64_t)r * E + e] = myv;
+        if (checker && one_rank && ld_cg(own + e) != myv) mismatch = true;  // the rank's own row
+    }
+    return mismatch;
+}
+
+// One rank's planning: the gathered counts must hold S*K non-negative picks
+// per rank, or the layout is undefined.  Every block checks every row (so all
+// take the same decision); block 0 copies the rows into the plan.
+__device__ __noinline__ void check_gathered_counts(const PlanArgs &a, int *s_cbad) {
+    const Dims &d = a.d;
+    const int E = d.E, R = d.R, lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    for (int q = w; q < R; q += kPlanWarps) {
+        const int32_t *row = a.counts_all + (int64_t)q * E;
+        long long sum = 0;
+        bool neg = false;
+        for (int e0 = 0; e0 < E; e0 += 32 * 8) {
+            int v[8];  // all loads of a batch in flight before any store
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int e = e0 + 32 * u + lane;
+                v[u] = e < E ? ld_cg(row + e) : 0;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int e = e0 + 32 * u + lane;
+                neg |= v[u] < 0;
+                sum += v[u];
+                if (blockIdx.x == 0 && e < E) a.plan.counts[(int64_t)q * E + e] = v[u];
+            }
+        }
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        const bool rowbad = __any_sync(0xffffffffu, neg) || sum != (long long)d.S * d.K;
+        if (lane == 0 && rowbad) atomicOr(s_cbad, MOONEP_STATUS_COUNT_MISMATCH);
+    }
+}
+
+// Block 0 of group planning: the router's local counts against the counts of
+// this call, every (rank, expert) once.  Run by the threads that have no
+// column-pass work, so it stays off the other threads' path; thread t of n
+// takes entries t, t + n, ..., 8 loads in flight per batch, so the check
+// costs one round of loads like the column pass beside it.
+__device__ __noinline__ bool check_router_counts(const PlanArgs &a, const int32_t *cnt, const int32_t *tpe_s,
+                                                 int t, int n) {
+    const Dims &d = a.d;
+    const int tot = d.R * d.E;
+    bool mismatch = false;
+    for (int i0 = t; i0 < tot; i0 += 8 * n) {
+        int v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = i0 + u * n;
+            v[u] = i < tot ? ld_cg(cnt + i) : 0;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = i0 + u * n;
+            if (i < tot && v[u] != (tpe_in_smem(d) ? tpe_s[i] : __ldg(a.tpe + i))) mismatch = true;
+        }
+    }
+    return mismatch;
+}
+
+// Mode 2: rank s takes into its B slots the received experts with the most
+// picks (ties to the lower index).  nrecv_s holds every received expert's
+// picks; expert j with ov picks is taken when fewer than B beat it.
+__device__ __noinline__ bool take_by_count(const int32_t *nrecv_s, int G, int j, int ov, int B) {
+    int better = 0;
+    for (int m = 0; m < G; ++m) {
+        const int om = nrecv_s[m];
+        better += (om > ov) || (om == ov && m < j);
+    }
+    return better < B;
+}
+
+// Fold this block's offset of each expert (its start in the group sequence
+// plus the picks of earlier chunks) into the kept-pick base and limit, so a
+// pick of rank rk inside the chunk needs only rk: its position in the group
+// sequence is g = off + rk.  T and pre are rewritten (the outputs never read
+// them).  Used when the layout tables have no room for the rank pass to do it.
+__device__ __noinline__ void fold_chunk_offsets(int32_t *T, int32_t *pre, const int32_t *es, const int32_t *pre2,
+                                                const int32_t *kbase, const int *s_keep, int E, int G, int t, int n) {
+    for (int e = t; e < E; e += n) {
+        const int off = es[e] + pre[e] + (pre2 ? pre2[e] : 0);
+        T[e] = kbase[e] + off;          // kept pick: dst = T[e] + rk ...
+        pre[e] = s_keep[e / G] - off;   // ... while rk < pre[e]
+    }
+}
+
 // ---- the planner kernel ----------------------------------------------------
 // 1024 threads per block: the register budget is 64 per thread.
-__global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
+__global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_constant__ PlanArgs a) {
     extern __shared__ __align__(16) uint8_t smem[];
     const Dims &d = a.d;
     const int E = d.E, K = d.K, R = d.R, G = d.G, B = d.B, NR = d.NR, tp = d.tp;
@@ -431,17 +582,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
             if (i < w1) ent_rank[i] = (uint16_t)(prior + before);
         }
     }
-    if (!whole_tokens) {  // tokens straddle runs: check duplicates token by token
-        for (int tt = tid; tt < t1 - t0; tt += kPlanThreads) {
-            const uint16_t *tok = ent_e + tt * K;
-            for (int k = 1; k < K; ++k) {
-                const uint16_t ek = tok[k];
-                if (ek == 0xFFFF) continue;
-                for (int k2 = 0; k2 < k; ++k2)
-                    if (tok[k2] == ek) bad |= MOONEP_STATUS_DUP_EXPERT;
-            }
-        }
-    }
+    if (!whole_tokens) bad |= dup_by_token(ent_e, t1 - t0, K);  // tokens straddle runs
     __syncthreads();
     PLAN_TRACE(7);
     // chunk totals: the histogram row (read back by this rank's later chunks)
@@ -545,6 +686,9 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
     const int col2 = 32 * (aw + 1);
     const bool colsplit = MOONEP_PLAN_COLSPLIT && d.xtab && col2 + E <= kPlanThreads;
     const bool foldrank = MOONEP_PLAN_FOLDRANK && d.xtab;
+    // the router-count check of block 0 runs on the threads past the split
+    // column pass when there is at least a warp of them
+    const bool spare_check = colsplit && kPlanThreads - (col2 + E) >= 32;
     if (!one_rank && w == aw) {
         for (int h = lane; h < R; h += 32) s_L[h] = ld_cg(a.ws.gload + (size_t)parity * R + h);
         __syncwarp();
@@ -570,7 +714,6 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
         const int32_t *mine_rows = a.ws.hist + (int64_t)r * d.nch * E;
         // rows q < R are the per-rank counts, rows R <= q < R + c this rank's
         // earlier chunk histograms; 16 loads in flight per batch
-        const int nrows = R + c;
         if (colsplit) {
             // warps 0.. sum the per-rank counts, the warps after the alias
             // warp this rank's earlier chunk rows: one batch of loads each
@@ -589,16 +732,15 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
                         tot += v[u];
                         if (q < r) mypre += v[u];
                         if (q == r) myv = v[u];
-                        if (checker && !one_rank) {
-                            const int t = tpe_in_smem(d) ? tpe_s[q * E + e] : __ldg(a.tpe + (int64_t)q * E + e);
-                            if (t != v[u]) mismatch = true;
-                        }
                     }
                 }
                 T[e] = tot;
                 pre[e] = mypre;
                 if (c == 0 && !one_rank) a.plan.counts[(int64_t)r * E + e] = myv;
                 if (checker && one_rank && ld_cg(own + e) != myv) mismatch = true;  // the rank's own row
+                if (checker && !one_rank && !spare_check) mismatch |= check_router_counts(a, cnt, tpe_s, e, E);
+            } else if (checker && !one_rank && spare_check && tid >= col2 + E) {
+                mismatch = check_router_counts(a, cnt, tpe_s, tid - (col2 + E), kPlanThreads - (col2 + E));
             } else if (tid >= col2 && tid < col2 + E) {
                 const int e = tid - col2;
                 int sum = 0;
@@ -612,37 +754,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
                 pre2[e] = sum;
             }
         } else {
-            for (int e = tid; e < E; e += kPlanThreads) {
-                int tot = 0, mypre = 0, myv = 0;
-                for (int q0 = 0; q0 < nrows; q0 += 16) {
-                    int v[16];
-#pragma unroll
-                    for (int u = 0; u < 16; ++u) {
-                        const int q = q0 + u;
-                        const int32_t *src = q < R ? cnt + (int64_t)q * E + e : mine_rows + (int64_t)(q - R) * E + e;
-                        v[u] = q < nrows ? ld_cg(src) : 0;
-                    }
-#pragma unroll
-                    for (int u = 0; u < 16; ++u) {
-                        const int q = q0 + u;
-                        if (q < R) {
-                            tot += v[u];
-                            if (q < r) mypre += v[u];
-                            if (q == r) myv = v[u];
-                            if (checker && !one_rank) {
-                                const int t = tpe_in_smem(d) ? tpe_s[q * E + e] : __ldg(a.tpe + (int64_t)q * E + e);
-                                if (t != v[u]) mismatch = true;
-                            }
-                        } else {
-                            mypre += v[u];  // 0 past the last row
-                        }
-                    }
-                }
-                T[e] = tot;
-                pre[e] = mypre;
-                if (c == 0 && !one_rank) a.plan.counts[(int64_t)r * E + e] = myv;
-                if (checker && one_rank && ld_cg(own + e) != myv) mismatch = true;  // the rank's own row
-            }
+            mismatch = column_pass_one_loop(a, cnt, own, mine_rows, tpe_s, T, pre, r, c, checker, one_rank);
         }
     }
     // the router's counts are checked by block 0 only, which writes the
@@ -657,31 +769,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
     // One rank: the gathered counts must hold S*K non-negative picks per rank,
     // or the layout below is undefined.  Every block checks every row, so all
     // take the same decision; block 0 copies the rows into the plan.
-    if (one_rank) {
-        for (int q = w; q < R; q += kPlanWarps) {
-            const int32_t *row = a.counts_all + (int64_t)q * E;
-            long long sum = 0;
-            bool neg = false;
-            for (int e0 = 0; e0 < E; e0 += 32 * 8) {
-                int v[8];  // all loads of a batch in flight before any store
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int e = e0 + 32 * u + lane;
-                    v[u] = e < E ? ld_cg(row + e) : 0;
-                }
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int e = e0 + 32 * u + lane;
-                    neg |= v[u] < 0;
-                    sum += v[u];
-                    if (blockIdx.x == 0 && e < E) a.plan.counts[(int64_t)q * E + e] = v[u];
-                }
-            }
-            for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-            const bool rowbad = __any_sync(0xffffffffu, neg) || sum != (long long)d.S * K;
-            if (lane == 0 && rowbad) atomicOr(&s_cbad, MOONEP_STATUS_COUNT_MISMATCH);
-        }
-    }
+    if (one_rank) check_gathered_counts(a, &s_cbad);
     // group loads and the largest count
     int mx = 0;
     for (int e = tid; e < E; e += kPlanThreads) mx = max(mx, T[e]);
@@ -785,14 +873,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
                 if (j < G) ov = max(0, min(es[e] + T[e], a1) - max(es[e], a0));
                 const unsigned has = __ballot_sync(0xffffffffu, ov > 0);
                 bool take = ov > 0 && nq + __popc(has & lanemask_lt()) < B;
-                if (by_count && ov > 0) {
-                    int better = 0;
-                    for (int m = 0; m < G; ++m) {
-                        const int om = nrecv[s * G + m];
-                        better += (om > ov) || (om == ov && m < j);
-                    }
-                    take = better < B;
-                }
+                if (by_count && ov > 0) take = take_by_count(nrecv + s * G, G, j, ov, B);
                 const unsigned tk = __ballot_sync(0xffffffffu, take);
                 // slot index of a taken expert; B marks an overflow row
                 const int q = take ? nslot + __popc(tk & lanemask_lt()) : B;
@@ -946,16 +1027,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
         const int t2 = tid - 32 * ow, n2 = kPlanThreads - 32 * ow;
         int32_t *kb = dbase, *kl = dlim;
         if (!foldrank) {
-            // Fold this block's offset of each expert (its start in the group
-            // sequence plus the picks of earlier chunks) into the kept-pick
-            // base and limit, so a pick of rank rk inside the chunk needs only
-            // rk: its position in the group sequence is g = off + rk.  The
-            // outputs never read the arrays rewritten here (T, pre).
-            for (int e = t2; e < E; e += n2) {
-                const int off = es[e] + pre[e] + (colsplit ? pre2[e] : 0);
-                T[e] = kbase[e] + off;           // kept pick: dst = T[e] + rk ...
-                pre[e] = s_keep[e / G] - off;    // ... while rk < pre[e]
-            }
+            fold_chunk_offsets(T, pre, es, colsplit ? pre2 : nullptr, kbase, s_keep, E, G, t2, n2);
             asm volatile("bar.sync 1, %0;" ::"r"(n2) : "memory");
             kb = T;
             kl = pre;
@@ -973,6 +1045,8 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(PlanArgs a) {
             } else if (d.fast2 && rk < eend2[e]) {
                 dst = ebase2[e] + rk;
             } else {  // the expert's donated run spans three or more recipients
+                // (in line: a call inside this loop slows every pass of it
+                // by more than the code it would move out)
                 const int h = e / G;
                 const int g = rk + s_keep[h] - kl[e];
                 int dest = -1;
