@@ -58,6 +58,7 @@ typedef struct CUstream_st *moonep_stream_t;
 #define MOONEP_ERR_ALIGN (-3)  /* a tensor pointer is not 16-byte aligned */
 #define MOONEP_ERR_CUDA (-4)   /* a CUDA runtime call failed (allocation or launch) */
 #define MOONEP_ERR_SIZE (-5)   /* a size argument is outside the supported range */
+#define MOONEP_ERR_DEVICE (-6) /* an operand is not memory of the handle's own GPU */
 
 /* device-side status bits, OR-ed into plan->status */
 #define MOONEP_STATUS_BAD_EXPERT 1     /* an expert id outside [0, E) (e.g. a -1 mask) */
@@ -259,7 +260,11 @@ MOONEP_API int moonep_reduce_grad(moonep_handle_t h, const moonep_plan_t *plan, 
  *   y_nvs   [R,NvS,Hp] bf16  output
  * Requires token_padding % 128 == 0 (a 128-row tile never spans two rows),
  * H % 64 == 0 and Hp % 256 == 0, else MOONEP_ERR_SIZE; pointers 16-byte
- * aligned.  A failed plan (plan->status != 0) computes nothing.
+ * aligned.  Every operand must be memory of the handle's own GPU: the kernel
+ * feeds its tiles through TMA into two-SM clusters, which never read another
+ * GPU's memory.  A pointer that CUDA reports on another device (a peer or
+ * IPC mapping) gives MOONEP_ERR_DEVICE before anything is launched.  A failed
+ * plan (plan->status != 0) computes nothing.
  */
 MOONEP_API int moonep_group_gemm(moonep_handle_t h, const moonep_plan_t *plan, const void *x_nvs,
                                  const void *weights, const void *pool, void *y_nvs, int64_t Hp,

@@ -89,6 +89,7 @@ extern "C" const char *moonep_error_string(int code) {
         case MOONEP_ERR_ALIGN: return "tensor pointer not 16-byte aligned";
         case MOONEP_ERR_CUDA: return "CUDA runtime call failed";
         case MOONEP_ERR_SIZE: return "size argument out of the supported range";
+        case MOONEP_ERR_DEVICE: return "operand not in the handle's own GPU memory";
         default: return "unknown moonep error";
     }
 }
@@ -485,6 +486,10 @@ extern "C" int moonep_group_gemm(moonep_handle_t h, const moonep_plan_t *plan, c
         return MOONEP_ERR_ALIGN;
     const int rc = gemm_supported(h->d, Hp);
     if (rc != MOONEP_OK) return rc;
+    // the GEMM reads its operands with TMA into two-SM clusters: local memory only
+    const void *ops[4] = {x_nvs, weights, pool, y_nvs};
+    for (const void *p : ops)
+        if (p && on_other_device(p, h->device) == 1) return MOONEP_ERR_DEVICE;
     int32_t *pairs = reinterpret_cast<int32_t *>(static_cast<char *>(h->ws_mem) + pair_table_offset(h->d));
     return launch_group_gemm(h->d, plan, x_nvs, weights, pool, y_nvs, Hp, pairs, reinterpret_cast<cudaStream_t>(stream));
 }

@@ -15,7 +15,7 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libmoonep.so")
 
-OK, ERR_NULL, ERR_CONFIG, ERR_ALIGN, ERR_CUDA, ERR_SIZE = 0, -1, -2, -3, -4, -5
+OK, ERR_NULL, ERR_CONFIG, ERR_ALIGN, ERR_CUDA, ERR_SIZE, ERR_DEVICE = 0, -1, -2, -3, -4, -5, -6
 STATUS_BAD_EXPERT, STATUS_DUP_EXPERT, STATUS_COUNT_MISMATCH, STATUS_BAD_PLAN, STATUS_TIMEOUT = 1, 2, 4, 8, 16
 MAX_R, MAX_E, MAX_K, MAX_PROJ = 64, 4096, 32, 8
 TRAINING, INFERENCE, INFERENCE_BY_COUNT, TRAINING_FEWEST_COPIES = 0, 1, 2, 3

@@ -42,6 +42,21 @@ def test_error_strings():
     assert moonep.error_string(0) == "ok"
 
 
+def test_every_error_code_is_bound_and_described():
+    # each MOONEP_ERR_* the header defines has the same value in the binding
+    # and a description of its own in the library
+    from load_balancing_planner_b200 import moonep
+    codes = dict(re.findall(r"#define MOONEP_(ERR_\w+)\s+\((-\d+)\)", open(HEADER).read()))
+    assert "ERR_DEVICE" in codes and len(codes) >= 6
+    texts = set()
+    for name, value in codes.items():
+        assert getattr(moonep, name) == int(value), name
+        text = moonep.error_string(int(value))
+        assert text != "unknown moonep error", name
+        texts.add(text)
+    assert len(texts) == len(codes)
+
+
 @pytest.mark.parametrize("bad", [
     dict(E=10, R=4),             # E % R != 0
     dict(K=9, E=8),              # K > E
