@@ -320,7 +320,7 @@ __device__ __noinline__ void expert_starts_by_count(const int32_t *T, int32_t *e
         for (int h = w - 1; w >= 1 && h < R; h += kPlanWarps - 1) {
             const int te = lane < G ? T[h * G + lane] : 0;
             int sum = 0;
-#pragma unroll 1
+#pragma unroll 8
             for (int m = 0; m < 32; ++m) {
                 const int tm = __shfl_sync(0xffffffffu, te, m);
                 sum += (m < G && (tm < te || (tm == te && m < lane))) ? tm : 0;
