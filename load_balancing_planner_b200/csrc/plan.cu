@@ -148,10 +148,9 @@ __device__ __forceinline__ int pad_to(int n, int tp) { return n ? (n + tp - 1) /
 // grid).  Both are called by every thread of the block.
 __device__ void grid_arrive(unsigned long long *ctr) {
     __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();
-        atomicAdd(ctr, 1ull);
-    }
+    // release at GPU scope: the block's writes ordered before it by the
+    // barrier above are visible to whoever acquires the counter
+    if (threadIdx.x == 0) asm volatile("red.release.gpu.global.add.u64 [%0], 1;" ::"l"(ctr) : "memory");
 }
 
 __device__ bool grid_wait(unsigned long long *ctr, unsigned long long target, uint32_t polls) {
@@ -159,15 +158,15 @@ __device__ bool grid_wait(unsigned long long *ctr, unsigned long long target, ui
     __syncthreads();
     if (threadIdx.x == 0) {
         int ok = 0;
-        const volatile unsigned long long *v = ctr;
         for (uint32_t it = 0; it < polls; ++it) {
-            if (*v >= target) {
+            unsigned long long v;
+            asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(ctr) : "memory");
+            if (v >= target) {
                 ok = 1;
                 break;
             }
             if (it > 64) __nanosleep(32);
         }
-        __threadfence();
         s_ok = ok;
     }
     __syncthreads();
@@ -509,6 +508,21 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
     const int CW = d.cw;
     uint16_t *wcnt = reinterpret_cast<uint16_t *>(region1);                       // [CW][E]
     uint32_t *wmask = reinterpret_cast<uint32_t *>(region1 + counts_bytes(d));    // [CW][E]
+    const int row = one_rank ? a.src_rank * d.nch + (int)blockIdx.x : (int)blockIdx.x;  // histogram row = r * nch + c
+    const int r = row / d.nch, c = row - r * d.nch;
+    const int t0 = c * d.ct;
+    const int t1 = min(d.S, t0 + d.ct);
+    const int n_ent = (t1 - t0) * K;
+    // picks (and their dst) of this chunk: [R,S,K] for the group, [S,K] for one rank
+    const int64_t base = ((one_rank ? 0 : (int64_t)r * d.S) + t0) * K;
+    // the chunk's first picks are loaded before the clears below, so their
+    // latency overlaps them
+    int pk[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        const int i = tid + u * kPlanThreads;
+        pk[u] = i < n_ent ? __ldg(a.topk + base + i) : 0;
+    }
     for (int i = tid; i < CW * E; i += kPlanThreads) {
         wcnt[i] = 0;
         wmask[i] = 0u;
@@ -529,17 +543,20 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
     }
 
     PLAN_TRACE(0);
-    const int row = one_rank ? a.src_rank * d.nch + (int)blockIdx.x : (int)blockIdx.x;  // histogram row = r * nch + c
-    const int r = row / d.nch, c = row - r * d.nch;
-    const int t0 = c * d.ct;
-    const int t1 = min(d.S, t0 + d.ct);
-    const int n_ent = (t1 - t0) * K;
-    // picks (and their dst) of this chunk: [R,S,K] for the group, [S,K] for one rank
-    const int64_t base = ((one_rank ? 0 : (int64_t)r * d.S) + t0) * K;
 
     // ---------------- A. count ----------------
     int bad = 0;
-    for (int i = tid; i < n_ent; i += kPlanThreads) {
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        const int i = tid + u * kPlanThreads;
+        if (i < n_ent) {
+            const int e = pk[u];
+            const bool good = e >= 0 && e < E;
+            if (!good) bad |= MOONEP_STATUS_BAD_EXPERT;
+            ent_e[i] = good ? (uint16_t)e : (uint16_t)0xFFFF;
+        }
+    }
+    for (int i = tid + 2 * kPlanThreads; i < n_ent; i += kPlanThreads) {
         const int e = __ldg(a.topk + base + i);
         const bool good = e >= 0 && e < E;
         if (!good) bad |= MOONEP_STATUS_BAD_EXPERT;
